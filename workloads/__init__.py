@@ -1,0 +1,216 @@
+"""Seeded synthetic inputs for the FP8 block-scaled GEMM, shared by the tests, the smoke check
+and the benchmark.
+
+This module holds no arithmetic of the GEMM itself.  It draws fp32 matrices from a seeded
+CPU generator and turns them into the inputs the method consumes: e4m3 codes plus one fp32
+scale per 1x128 tile of A and per 128x128 block of B (the DeepSeek-V3 fine-grained scaling
+that the DeepGEMM write-up names in "深入了解DeepGEMM").  The scale of a tile is its
+absolute maximum divided by 448 (the largest finite e4m3 magnitude), clamped away from zero;
+the code is the tile divided by its scale, cast to e4m3 with round-to-nearest-even by torch.
+Both the oracle and the CUDA library consume the same codes and scales, so this step does not
+enter the parity comparison.
+
+Every array returned here is a CPU numpy/torch array in the LOGICAL layout:
+  a codes [rows, K] uint8, sa [rows, K/128] float32,
+  b codes [N, K] uint8 (grouped: [G, N, K]), sb [ceil(N/128), K/128] (grouped: [G, ...]).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+BLOCK = 128
+E4M3_MAX = 448.0
+AMAX_FLOOR = 1e-4
+
+
+def _gen(seed: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return g
+
+
+def quantise_rows_1x128(x: torch.Tensor):
+    """fp32 [R, K] -> (codes uint8 [R, K], scales fp32 [R, K/128]); one scale per 1x128 tile."""
+    R, K = x.shape
+    assert K % BLOCK == 0
+    t = x.float().reshape(R, K // BLOCK, BLOCK)
+    amax = t.abs().amax(dim=2).clamp_min(AMAX_FLOOR)
+    scale = (amax / E4M3_MAX).float()
+    codes = (t / scale.unsqueeze(2)).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.reshape(R, K).numpy(), scale.numpy()
+
+
+def quantise_blocks_128x128(x: torch.Tensor):
+    """fp32 [N, K] -> (codes uint8 [N, K], scales fp32 [ceil(N/128), K/128]); one scale per
+    128x128 block (a partial last block of rows gets its own scale over its real rows)."""
+    N, K = x.shape
+    assert K % BLOCK == 0
+    Nb, Kb = -(-N // BLOCK), K // BLOCK
+    pad = Nb * BLOCK - N
+    xp = torch.nn.functional.pad(x.float(), (0, 0, 0, pad)) if pad else x.float()
+    t = xp.reshape(Nb, BLOCK, Kb, BLOCK)
+    amax = t.abs().amax(dim=(1, 3)).clamp_min(AMAX_FLOOR)
+    scale = (amax / E4M3_MAX).float()
+    q = (t / scale[:, None, :, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    codes = q.reshape(Nb * BLOCK, K)[:N]
+    return codes.contiguous().numpy(), scale.numpy()
+
+
+@dataclass
+class Dense:
+    M: int
+    N: int
+    K: int
+    a: np.ndarray
+    sa: np.ndarray
+    b: np.ndarray
+    sb: np.ndarray
+
+    @property
+    def flops(self) -> float:
+        return 2.0 * self.M * self.N * self.K
+
+
+@dataclass
+class Contiguous:
+    G: int
+    N: int
+    K: int
+    counts: np.ndarray          # valid rows per expert
+    m_indices: np.ndarray       # int32 [M_total], expert or -1
+    a: np.ndarray               # [M_total, K]
+    sa: np.ndarray              # [M_total, K/128]
+    b: np.ndarray               # [G, N, K]
+    sb: np.ndarray              # [G, ceil(N/128), K/128]
+
+    @property
+    def M_total(self) -> int:
+        return int(self.a.shape[0])
+
+    @property
+    def flops(self) -> float:
+        return 2.0 * float(self.counts.sum()) * self.N * self.K
+
+
+@dataclass
+class Masked:
+    G: int
+    M_max: int
+    N: int
+    K: int
+    expected_m: int
+    masked_m: np.ndarray        # int32 [G]
+    a: np.ndarray               # [G, M_max, K]
+    sa: np.ndarray              # [G, M_max, K/128]
+    b: np.ndarray               # [G, N, K]
+    sb: np.ndarray              # [G, ceil(N/128), K/128]
+
+    @property
+    def flops(self) -> float:
+        return 2.0 * float(self.masked_m.sum()) * self.N * self.K
+
+
+def dense(M: int, N: int, K: int, seed: int, a_std: float = 1.0, b_std: float = 1.0,
+          outlier_frac: float = 0.0, outlier_scale: float = 50.0) -> Dense:
+    """A ~ N(0, a_std^2) [M,K], B ~ N(0, b_std^2) [N,K]; draw order A, B, then (if
+    outlier_frac > 0) an independent Bernoulli(outlier_frac) mask over A whose elements are
+    multiplied by outlier_scale before quantisation."""
+    g = _gen(seed)
+    A = torch.randn(M, K, generator=g) * a_std
+    B = torch.randn(N, K, generator=g) * b_std
+    if outlier_frac > 0:
+        mask = torch.rand(M, K, generator=g) < outlier_frac
+        A = torch.where(mask, A * outlier_scale, A)
+    a, sa = quantise_rows_1x128(A)
+    b, sb = quantise_blocks_128x128(B)
+    return Dense(M, N, K, a, sa, b, sb)
+
+
+def _grouped_b(G: int, N: int, K: int, std: float, g: torch.Generator):
+    Nb, Kb = -(-N // BLOCK), K // BLOCK
+    b = np.empty((G, N, K), np.uint8)
+    sb = np.empty((G, Nb, Kb), np.float32)
+    for e in range(G):
+        be, se = quantise_blocks_128x128(torch.randn(N, K, generator=g) * std)
+        b[e], sb[e] = be, se
+    return b, sb
+
+
+def contiguous(G: int, N: int, K: int, seed: int, count_lo: int = 128, count_hi: int = 1024,
+               a_std: float = 1.0, b_std: float = 0.02, counts=None) -> Contiguous:
+    """Per-expert token counts uniform in [count_lo, count_hi] (inclusive), each segment padded
+    up to a multiple of 128 with rows whose expert index is -1.  Draw order: counts, A (all
+    rows, padding included), B per expert."""
+    g = _gen(seed)
+    if counts is None:
+        counts = torch.randint(count_lo, count_hi + 1, (G,), generator=g).numpy()
+    counts = np.asarray(counts, dtype=np.int64)
+    padded = (counts + BLOCK - 1) // BLOCK * BLOCK
+    M_total = int(padded.sum())
+    m_idx = np.full(M_total, -1, np.int32)
+    off = 0
+    for e in range(G):
+        m_idx[off:off + counts[e]] = e
+        off += int(padded[e])
+    A = torch.randn(M_total, K, generator=g) * a_std
+    a, sa = quantise_rows_1x128(A)
+    b, sb = _grouped_b(G, N, K, b_std, g)
+    return Contiguous(G, N, K, counts, m_idx, a, sa, b, sb)
+
+
+def masked(G: int, M_max: int, N: int, K: int, seed: int, expected_m: int = 128,
+           a_std: float = 1.0, b_std: float = 0.02, masked_m=None) -> Masked:
+    """masked_m[g] uniform in [0, M_max] (inclusive); every row of A is filled, valid or not.
+    Draw order: masked_m, A, B per expert."""
+    g = _gen(seed)
+    if masked_m is None:
+        masked_m = torch.randint(0, M_max + 1, (G,), generator=g).numpy()
+    masked_m = np.asarray(masked_m, dtype=np.int32)
+    A = torch.randn(G * M_max, K, generator=g) * a_std
+    a, sa = quantise_rows_1x128(A)
+    a = a.reshape(G, M_max, K)
+    sa = sa.reshape(G, M_max, K // BLOCK)
+    b, sb = _grouped_b(G, N, K, b_std, g)
+    return Masked(G, M_max, N, K, expected_m, masked_m, a, sa, b, sb)
+
+
+# ---- the named workloads ----------------------------------------------------------------
+
+SMALL_DENSE = dict(M=128, N=256, K=512)
+SWEEP_NK = [(2112, 7168), (24576, 1536), (7168, 16384), (4096, 7168), (7168, 2048)]
+SWEEP_M = [64, 128, 4096]
+CONTIG = dict(G=8, N=4096, K=7168)
+MASKED = dict(G=32, M_max=256, N=4096, K=7168, expected_m=128)
+PREFILL = dict(M=8192, N=7168, K=18432)
+
+
+def small_dense(seed: int = 1000) -> Dense:
+    """128x256x512, A and B ~ N(0,1)."""
+    return dense(**SMALL_DENSE, seed=seed)
+
+
+def sweep_shapes():
+    """The fifteen (M, N, K) shapes of the dense sweep, M-major."""
+    return [(m, n, k) for m in SWEEP_M for (n, k) in SWEEP_NK]
+
+
+def sweep_case(i: int) -> Dense:
+    """Shape i of the dense sweep: A ~ N(0,1), B ~ N(0, 0.02^2)."""
+    M, N, K = sweep_shapes()[i]
+    return dense(M, N, K, seed=2000 + i, a_std=1.0, b_std=0.02)
+
+
+def contiguous_case(seed: int = 3000) -> Contiguous:
+    return contiguous(**CONTIG, seed=seed)
+
+
+def masked_case(seed: int = 4000) -> Masked:
+    return masked(**MASKED, seed=seed)
+
+
+def prefill_case(seed: int = 5000) -> Dense:
+    """8192x7168x18432 with ~1% outliers x50 in A."""
+    return dense(**PREFILL, seed=seed, a_std=1.0, b_std=0.02, outlier_frac=0.01)
