@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Benchmark of the FP8 block-scaled NT GEMM library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload sweep|small|contiguous|masked|prefill]
+
+Prints ONE JSON line on rank 0.  A "step" is one pass of the whole hot path over one batch of
+synthetic input: for the default workload, the fifteen GEMMs of the dense sweep
+(M in {64, 128, 4096} x (N, K) in {(2112,7168), (24576,1536), (7168,16384), (4096,7168),
+(7168,2048)}; A ~ N(0,1), B ~ N(0,0.02^2), fp32 scales per 1x128 tile of A and per 128x128
+block of B).  Inputs are resident in HBM; CUDA events bracket every GEMM on the launching
+stream, and the step is enqueued behind a bounded sleep kernel so that host latency never
+falls inside a bracket.  L2 is flushed (a 256 MiB write) before every step, and the step's own working set
+exceeds L2.
+
+`value` is the aggregate FP8 TFLOPS of the step (sum of 2*M*N*K over its GEMMs / sum of their
+device times), summed over ranks (each rank runs its own copy of the step: weak scaling, no
+collective on the data path).  `e2e` is the same metric through the Python binding with host
+buffers: pinned host -> device copies of every input, the GEMMs, and the device -> host copy of
+every output inside the timed region.  `--impl reference` times the CPU oracle on a bounded
+sample of the same workload on this machine's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "FP8 TFLOPS and GB/s per shape at 1 B200; fraction of FP8-peak/HBM roofline"
+UNIT = "TFLOPS"
+L2_FLUSH_BYTES = 256 << 20
+FP8_PER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor ratio on B200 (4.5 / 2.25 PFLOP/s)
+
+
+# ---- workload description ---------------------------------------------------------------------
+
+class Gemm:
+    """One GEMM of a step: its kind, sizes, FLOPs and algorithmic bytes."""
+
+    def __init__(self, kind: str, case, name: str):
+        self.kind, self.case, self.name = kind, case, name
+        c = case
+        if kind == "dense":
+            M, N, K, groups, m_valid, m_rows = c.M, c.N, c.K, 1, c.M, c.M
+        elif kind == "contiguous":
+            M, N, K = c.M_total, c.N, c.K
+            m_valid, m_rows = int(c.counts.sum()), c.M_total
+            groups = int(np.count_nonzero(c.counts))
+        else:
+            M, N, K = c.M_max, c.N, c.K
+            m_valid, m_rows = int(c.masked_m.sum()), int(c.masked_m.sum())
+            groups = int(np.count_nonzero(c.masked_m))
+        kb, nb = K // 128, -(-N // 128)
+        self.flops = 2.0 * m_valid * N * K
+        # each operand once: A rows that are computed, B of every group touched, D, the scales,
+        # and the int32 row indices of the contiguous layout
+        self.bytes = (m_valid * K + N * K * groups + 2 * m_valid * N + 4 * m_rows * kb
+                      + 4 * nb * kb * groups + (4 * M if kind == "contiguous" else 0))
+        self.shape = dict(kind=kind, M=M, N=N, K=K, G=getattr(c, "G", 1), M_valid=m_valid)
+
+
+def build_workload(name: str):
+    if name == "sweep":
+        gemms = []
+        for i, (M, N, K) in enumerate(workloads.sweep_shapes()):
+            gemms.append(Gemm("dense", workloads.sweep_case(i), f"dense {M}x{N}x{K}"))
+        desc = ("dense FP8 NT GEMM sweep, M in {64,128,4096} x (N,K) in {(2112,7168),(24576,1536),"
+                "(7168,16384),(4096,7168),(7168,2048)}; A~N(0,1), B~N(0,0.02); fp32 scales per 1x128 "
+                "A tile and 128x128 B block; bf16 out")
+        return gemms, desc
+    if name == "small":
+        c = workloads.small_dense()
+        return [Gemm("dense", c, "dense 128x256x512")], "dense FP8 NT GEMM M=128 N=256 K=512, A,B~N(0,1)"
+    if name == "contiguous":
+        c = workloads.contiguous_case()
+        return [Gemm("contiguous", c, f"contiguous G=8 M_total={c.M_total} N=4096 K=7168")], \
+            ("contiguous grouped MoE GEMM, G=8, per-expert counts U[128,1024] padded to 128, "
+             "N=4096, K=7168, B~N(0,0.02)")
+    if name == "masked":
+        c = workloads.masked_case()
+        return [Gemm("masked", c, "masked G=32 M_max=256 N=4096 K=7168")], \
+            ("masked grouped MoE GEMM, G=32, M_max=256, masked_m U[0,256], expected_m=128, "
+             "N=4096, K=7168, B~N(0,0.02)")
+    if name == "prefill":
+        c = workloads.prefill_case()
+        return [Gemm("dense", c, "dense 8192x7168x18432")], \
+            "dense FP8 NT GEMM M=8192 N=7168 K=18432, A~N(0,1) with 1% x50 outliers, B~N(0,0.02)"
+    raise SystemExit(f"unknown workload {name}")
+
+
+# ---- peaks and roofline ---------------------------------------------------------------------------
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16_tflops=float(p["bf16_tflops"]),
+                    bf16_tflops_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def roofline(g: Gemm, seconds: float, peaks) -> dict:
+    fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16 * 1e12
+    bw = peaks["hbm_gbs"] * 1e9
+    t_flop, t_mem = g.flops / fp8_peak, g.bytes / bw
+    bound = "tensor" if t_flop >= t_mem else "hbm"
+    return dict(name=g.name, **g.shape, us=seconds * 1e6, tflops=g.flops / seconds / 1e12,
+                gbs=g.bytes / seconds / 1e9, bound=bound, roof_us=max(t_flop, t_mem) * 1e6,
+                frac=max(t_flop, t_mem) / seconds)
+
+
+# ---- clocks ---------------------------------------------------------------------------------------
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a background thread."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
+               0x2: "applications_clocks_setting", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+                mask = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return dict(sm_mhz=None, sm_max_mhz=self.max_mhz, reasons=sorted(self.reasons), samples=0)
+        return dict(sm_mhz=float(statistics.median(self.samples)), sm_max_mhz=self.max_mhz,
+                    reasons=sorted(self.reasons - {"gpu_idle"}), samples=len(self.samples))
+
+
+# ---- our arm ------------------------------------------------------------------------------------
+
+class DeviceGemm:
+    """Device-resident inputs and output of one GEMM, and the launch through the binding."""
+
+    def __init__(self, dg, g: Gemm):
+        self.g = g
+        c = g.case
+        self.a = torch.from_numpy(np.ascontiguousarray(c.a)).cuda()
+        self.b = torch.from_numpy(np.ascontiguousarray(c.b)).cuda()
+        self.sfa = dg.sfa_mn_major(torch.from_numpy(c.sa).cuda())
+        self.sfb = torch.from_numpy(c.sb).cuda()
+        self.extra = None
+        if g.kind == "dense":
+            self.d = torch.empty(c.M, c.N, dtype=torch.bfloat16, device="cuda")
+        elif g.kind == "contiguous":
+            self.d = torch.empty(c.M_total, c.N, dtype=torch.bfloat16, device="cuda")
+            self.extra = torch.from_numpy(c.m_indices).cuda()
+        else:
+            self.d = torch.empty(c.G, c.M_max, c.N, dtype=torch.bfloat16, device="cuda")
+            self.extra = torch.from_numpy(c.masked_m).cuda()
+        self.dg = dg
+
+    def tensors_in(self):
+        t = [self.a, self.sfa, self.b, self.sfb]
+        if self.extra is not None:
+            t.append(self.extra)
+        return t
+
+    def launch(self, stream=None):
+        dg, c = self.dg, self.g.case
+        if self.g.kind == "dense":
+            dg.dg_gemm_fp8_fp8_bf16_nt(self.a, self.sfa, self.b, self.sfb, self.d, stream=stream)
+        elif self.g.kind == "contiguous":
+            dg.dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(self.a, self.sfa, self.b, self.sfb,
+                                                            self.d, self.extra, stream=stream)
+        else:
+            dg.dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked(self.a, self.sfa, self.b, self.sfb, self.d,
+                                                        self.extra, c.expected_m, stream=stream)
+
+
+def run_ours(args, rank, world, local_rank):
+    import fp8_block_scaled_tma_b200 as dg
+
+    torch.cuda.set_device(local_rank)
+    gemms, desc = build_workload(args.workload)
+    dev = [DeviceGemm(dg, g) for g in gemms]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    n = len(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+    gate = [2_000_000]  # GPU cycles the stream is held so the host can enqueue the whole step
+
+    def step():
+        # a bounded sleep kernel holds the stream while the host enqueues the step, so no host
+        # latency falls between an event and the GEMM it brackets; then the L2 flush
+        torch.cuda._sleep(gate[0])
+        flush.fill_(1)
+        t0 = time.perf_counter()
+        for i, d in enumerate(dev):
+            ev[i].record(stream)
+            d.launch(stream)
+        ev[n].record(stream)
+        host = time.perf_counter() - t0
+        stream.synchronize()
+        if host * 1.9e9 * 1.5 > gate[0]:
+            gate[0] = int(host * 1.9e9 * 3)
+        return [ev[i].elapsed_time(ev[i + 1]) * 1e-3 for i in range(n)]
+
+    for _ in range(args.warmup):
+        step()
+    launch_info = dg.get_last_launch()
+    if dg.poll_device_error(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+
+    per = [[] for _ in range(n)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for _ in range(args.steps):
+            for i, s in enumerate(step()):
+                per[i].append(s)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    total = sum(sum(p) for p in per)  # device seconds over the timed steps
+    t = torch.tensor([total], dtype=torch.float64, device="cuda")
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_max = float(t.item())
+    if dg.poll_device_error(stream) != 0:
+        raise RuntimeError("device error during the timed steps")
+
+    flops_step = sum(g.flops for g in gemms)
+    bytes_step = sum(g.bytes for g in gemms)
+    value = world * flops_step * args.steps / total_max / 1e12
+    peaks = load_peaks()
+    shapes = [roofline(g, statistics.mean(p), peaks) for g, p in zip(gemms, per)]
+    dom = max(range(n), key=lambda i: sum(per[i]))
+    dsh = shapes[dom]
+    if dsh["bound"] == "tensor":
+        peak = peaks["bf16_tflops"] * FP8_PER_BF16
+        roof = dict(bound="tensor", achieved=dsh["tflops"], peak=peak, unit="TFLOP/s",
+                    frac=dsh["tflops"] / peak,
+                    peak_source=f"{peaks['source']} bf16 burst x{FP8_PER_BF16:g} (nominal FP8/BF16 ratio)")
+    else:
+        peak = peaks["hbm_gbs"]
+        roof = dict(bound="hbm", achieved=dsh["gbs"], peak=peak, unit="GB/s",
+                    frac=dsh["gbs"] / peak, peak_source=f"{peaks['source']} HBM copy")
+    roof.update(kernel=dsh["name"], traffic=args.traffic_bytes, traffic_unit="bytes/launch")
+
+    out = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps,
+               warmup=args.warmup, ms_per_step=total_max / args.steps * 1e3,
+               higher_is_better=True, scaling="weak", vs_baseline=None, dtype="e4m3 x e4m3 -> f32",
+               data="synthetic",
+               config=dict(workload=desc, gemms_per_step=n,
+                           l2="256 MiB write before every step; step working set > L2 (126 MB)",
+                           timing="CUDA events around each GEMM on the launching stream; the "
+                                  "step is enqueued behind a bounded sleep kernel",
+                           parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+               gbs=world * bytes_step * args.steps / total_max / 1e9,
+               roofline=roof, per_shape=shapes, gpu_launches=n * args.steps,
+               clocks=clk.summary(), last_launch=launch_info)
+
+    # e2e through the public API with host buffers
+    if not args.no_e2e:
+        out["e2e"] = run_e2e(dg, dev, gemms, args, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(gemms, budget_s=args.cpu_seconds)
+    return out
+
+
+def run_e2e(dg, dev, gemms, args, world):
+    """Host buffers -> device, the GEMMs through the binding, outputs -> host, per step."""
+    host_in = [[t.cpu().pin_memory() for t in d.tensors_in()] for d in dev]
+    host_out = [torch.empty(d.d.shape, dtype=d.d.dtype).pin_memory() for d in dev]
+    h2d = sum(t.numel() * t.element_size() for ts in host_in for t in ts)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def step():
+        e0.record(stream)
+        for d, hs, ho in zip(dev, host_in, host_out):
+            for dst, src in zip(d.tensors_in(), hs):
+                dst.copy_(src, non_blocking=True)
+            d.launch()
+            ho.copy_(d.d, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) * 1e-3
+
+    for _ in range(min(args.warmup, 3)):
+        step()
+    steps = max(1, min(args.steps, 10))
+    ts = [step() for _ in range(steps)]
+    t = torch.tensor([sum(ts)], dtype=torch.float64, device="cuda")
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    flops = sum(g.flops for g in gemms)
+    return dict(value=world * flops * steps / float(t.item()) / 1e12, unit=UNIT,
+                h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, steps=steps,
+                ms_per_step=float(t.item()) / steps * 1e3)
+
+
+# ---- CPU oracle (baseline and reference arm) --------------------------------------------------
+
+def _oracle_rows(g: Gemm, rows_per_gemm: int, rng):
+    import oracle
+    c = g.case
+    if g.kind == "dense":
+        r = np.sort(rng.choice(c.M, size=min(c.M, rows_per_gemm), replace=False))
+        oracle.gemm_dense(c.a, c.sa, c.b, c.sb, rows=r)
+        return 2.0 * len(r) * c.N * c.K
+    if g.kind == "contiguous":
+        valid = np.nonzero(c.m_indices >= 0)[0]
+        r = np.sort(rng.choice(valid, size=min(len(valid), rows_per_gemm), replace=False))
+        oracle.gemm_contiguous(c.a, c.sa, c.b, c.sb, c.m_indices, rows=r)
+        return 2.0 * len(r) * c.N * c.K
+    flat = np.array([gi * c.M_max + r for gi in range(c.G) for r in range(int(c.masked_m[gi]))])
+    r = np.sort(rng.choice(flat, size=min(len(flat), rows_per_gemm), replace=False))
+    oracle.gemm_masked(c.a, c.sa, c.b, c.sb, c.masked_m, rows=r)
+    return 2.0 * len(r) * c.N * c.K
+
+
+def oracle_sample_step(gemms, rows_per_gemm: int, rng) -> float:
+    return sum(_oracle_rows(g, rows_per_gemm, rng) for g in gemms)
+
+
+def cpu_baseline(gemms, budget_s: float = 15.0):
+    """The oracle as it stands, on this host's cores, over seeded random rows of every GEMM of
+    the step, repeated until about `budget_s` seconds of CPU work."""
+    import oracle
+    oracle.build()
+    cores = os.cpu_count() or 1
+    rows = max(16, cores)
+    rng = np.random.default_rng(1234)
+    flops, t0, passes = 0.0, time.perf_counter(), 0
+    while True:
+        flops += oracle_sample_step(gemms, rows, rng)
+        passes += 1
+        if time.perf_counter() - t0 >= budget_s or passes >= 50:
+            break
+    dt = time.perf_counter() - t0
+    return dict(value=flops / dt / 1e12, unit=UNIT, cores=cores, kind="oracle",
+                sample=f"{passes} pass(es) of {rows} seeded random rows of every GEMM of the step "
+                       f"({flops / 1e9:.1f} GFLOP in {dt:.1f} s, fp64, {cores} threads)")
+
+
+def run_reference(args):
+    """The CPU oracle on a bounded sample of the workload (rank 0 only)."""
+    import oracle
+    oracle.build()
+    gemms, desc = build_workload(args.workload)
+    cores = os.cpu_count() or 1
+    rows = 16
+    rng = np.random.default_rng(99)
+    for _ in range(args.warmup):
+        oracle_sample_step(gemms, rows, rng)
+    t0 = time.perf_counter()
+    flops = 0.0
+    for _ in range(args.steps):
+        flops += oracle_sample_step(gemms, rows, rng)
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    sample = f"{rows} seeded random rows of every GEMM of the step per step"
+    return dict(metric=METRIC, value=value, unit=UNIT, n_gpus=1, steps=args.steps,
+                warmup=args.warmup, ms_per_step=dt / args.steps * 1e3, higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
+                config=dict(workload=desc), impl="reference",
+                cpu_baseline=dict(value=value, unit=UNIT, cores=cores, kind="oracle", sample=sample),
+                e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+
+
+# ---- main ---------------------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["sweep", "small", "contiguous", "masked", "prefill"],
+                    default="sweep")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--traffic-bytes", type=float, default=None,
+                    help="dram bytes per launch of the dominant kernel from an ncu capture")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,249 @@
+"""Python binding of the B200 (sm_100a) FP8 block-scaled NT GEMM library.
+
+Argument marshalling only: each function checks shapes and dtypes of torch tensors and calls
+the C ABI of ``libdg_b200.so`` (declared in ``include/dg.h``) with their device pointers and
+the current CUDA stream.  Every step of the computation runs in the library's CUDA kernels;
+there is no fallback.  Importing this package fails loudly when the library is not built.
+
+Entry points (the names of the DeepGEMM release write-up, "如何使用"):
+  dg_gemm_fp8_fp8_bf16_nt                        dense NT GEMM
+  dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous   MoE grouped GEMM, contiguous layout
+  dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked       MoE grouped GEMM, masked layout
+plus the SM-count and TMA-alignment utilities.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdg_b200.so")
+
+DG_OK = 0
+DG_ERR_INVALID_ARG = -1
+DG_ERR_UNSUPPORTED = -2
+DG_ERR_CUDA = -3
+DG_ERR_TIMEOUT = -4
+DG_ERR_WORKSPACE = -5
+DG_ERR_LAYOUT = -6
+
+BLOCK = 128
+
+
+class DGError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build the CUDA library first "
+            "(python fp8_block_scaled_tma_b200/build.py, or __graft_entry__.build())")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, fp, ip, i, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.dg_gemm_fp8_fp8_bf16_nt.argtypes = [vp, fp, vp, fp, vp, i, i, i, vp, sz, vp]
+    lib.dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous.argtypes = [vp, fp, vp, fp, vp, ip, i, i, i,
+                                                                 i, vp, sz, vp]
+    lib.dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked.argtypes = [vp, fp, vp, fp, vp, ip, i, i, i, i,
+                                                             i, vp, sz, vp]
+    for name in ("dg_gemm_fp8_fp8_bf16_nt", "dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous",
+                 "dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked"):
+        getattr(lib, name).restype = ctypes.c_int
+    lib.dg_set_num_sms.argtypes = [i]
+    lib.dg_set_num_sms.restype = i
+    lib.dg_get_num_sms.argtypes = []
+    lib.dg_get_num_sms.restype = i
+    lib.dg_get_tma_aligned_size.argtypes = [i, i]
+    lib.dg_get_tma_aligned_size.restype = i
+    lib.dg_get_workspace_size.argtypes = [i, i, i, i, i]
+    lib.dg_get_workspace_size.restype = sz
+    lib.dg_status_string.argtypes = [i]
+    lib.dg_status_string.restype = ctypes.c_char_p
+    lib.dg_poll_device_error.argtypes = [vp]
+    lib.dg_poll_device_error.restype = i
+    lib.dg_set_wait_timeout_ns.argtypes = [ctypes.c_ulonglong]
+    lib.dg_set_wait_timeout_ns.restype = ctypes.c_ulonglong
+    lib.dg_set_config_override.argtypes = [i, i]
+    lib.dg_set_config_override.restype = i
+    ipp = ctypes.POINTER(ctypes.c_int)
+    lib.dg_get_last_launch.argtypes = [ipp, ipp, ipp, ipp]
+    lib.dg_get_last_launch.restype = i
+    return lib
+
+
+lib = _load()
+
+
+# ---- helpers ------------------------------------------------------------------------------
+
+def status_string(status: int) -> str:
+    return lib.dg_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != DG_OK:
+        raise DGError(status, where)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _fp8(t: torch.Tensor, name: str) -> None:
+    if t.dtype not in (torch.uint8, torch.float8_e4m3fn):
+        raise TypeError(f"{name} must hold e4m3 codes (uint8 or float8_e4m3fn), got {t.dtype}")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+def _f32(t: torch.Tensor, name: str, shape) -> None:
+    if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous float32 CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _out(t: torch.Tensor, shape) -> None:
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError("d must be a contiguous bfloat16 CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"d has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _i32(t: torch.Tensor, name: str, shape) -> None:
+    if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def get_tma_aligned_size(x: int, elem_bytes: int) -> int:
+    r = lib.dg_get_tma_aligned_size(int(x), int(elem_bytes))
+    if r < 0:
+        raise DGError(r, "dg_get_tma_aligned_size")
+    return r
+
+
+def set_num_sms(n: int) -> int:
+    return lib.dg_set_num_sms(int(n))
+
+
+def get_num_sms() -> int:
+    r = lib.dg_get_num_sms()
+    if r < 0:
+        raise DGError(r, "dg_get_num_sms")
+    return r
+
+
+def get_workspace_size(kind: int, M: int, N: int, K: int, G: int = 1) -> int:
+    return int(lib.dg_get_workspace_size(kind, M, N, K, G))
+
+
+def poll_device_error(stream=None) -> int:
+    return lib.dg_poll_device_error(_stream(stream))
+
+
+def set_wait_timeout_ns(ns: int) -> int:
+    return int(lib.dg_set_wait_timeout_ns(int(ns)))
+
+
+def set_config_override(block_n: int = 0, num_stages: int = 0) -> None:
+    _check(lib.dg_set_config_override(int(block_n), int(num_stages)), "dg_set_config_override")
+
+
+def get_last_launch() -> dict:
+    v = [ctypes.c_int() for _ in range(4)]
+    _check(lib.dg_get_last_launch(*[ctypes.byref(x) for x in v]), "dg_get_last_launch")
+    return dict(block_n=v[0].value, stages=v[1].value, grid=v[2].value, tiles=v[3].value)
+
+
+def sfa_mn_major(sa: torch.Tensor) -> torch.Tensor:
+    """Layout marshalling of A's scales: logical [rows, K/128] (or [G, rows, K/128]) fp32 ->
+    the MN-major, TMA-aligned layout the kernels read: [K/128, align4(rows)] (or
+    [G, K/128, align4(rows)]), zero in the padding."""
+    sa = sa.float()
+    if sa.dim() == 2:
+        rows, kb = sa.shape
+        out = torch.zeros(kb, get_tma_aligned_size(rows, 4), dtype=torch.float32, device=sa.device)
+        out[:, :rows] = sa.t()
+        return out
+    if sa.dim() == 3:
+        g, rows, kb = sa.shape
+        out = torch.zeros(g, kb, get_tma_aligned_size(rows, 4), dtype=torch.float32,
+                          device=sa.device)
+        out[:, :, :rows] = sa.transpose(1, 2)
+        return out
+    raise ValueError("sa must be 2-D or 3-D")
+
+
+# ---- the three GEMMs ------------------------------------------------------------------------
+
+def dg_gemm_fp8_fp8_bf16_nt(a, sfa, b, sfb, d, workspace=None, stream=None) -> None:
+    """d[M,N] (bf16) = a[M,K] (e4m3) . b[N,K]^T with sfa [K/128, align4(M)] (MN-major) and
+    sfb [ceil(N/128), K/128]."""
+    _fp8(a, "a")
+    _fp8(b, "b")
+    M, K = a.shape
+    N = b.shape[0]
+    if b.shape[1] != K:
+        raise ValueError("a and b disagree on K")
+    _f32(sfa, "sfa", (K // BLOCK, get_tma_aligned_size(M, 4)))
+    _f32(sfb, "sfb", (-(-N // BLOCK), K // BLOCK))
+    _out(d, (M, N))
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.dg_gemm_fp8_fp8_bf16_nt(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K,
+                                       _ptr(workspace), ws, _stream(stream)),
+           "dg_gemm_fp8_fp8_bf16_nt")
+
+
+def dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(a, sfa, b, sfb, d, m_indices, workspace=None,
+                                                 stream=None) -> None:
+    """Contiguous-layout grouped GEMM: a [M_total,K], sfa [K/128, M_total], b [G,N,K],
+    sfb [G, ceil(N/128), K/128], d [M_total,N], m_indices int32 [M_total] (-1 = padding)."""
+    _fp8(a, "a")
+    _fp8(b, "b")
+    M, K = a.shape
+    G, N, Kb_ = b.shape
+    if Kb_ != K:
+        raise ValueError("a and b disagree on K")
+    _f32(sfa, "sfa", (K // BLOCK, get_tma_aligned_size(M, 4)))
+    _f32(sfb, "sfb", (G, -(-N // BLOCK), K // BLOCK))
+    _out(d, (M, N))
+    _i32(m_indices, "m_indices", (M,))
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(
+        _ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), _ptr(m_indices), M, N, K, G,
+        _ptr(workspace), ws, _stream(stream)), "dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous")
+
+
+def dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked(a, sfa, b, sfb, d, masked_m, expected_m: int,
+                                             workspace=None, stream=None) -> None:
+    """Masked-layout grouped GEMM: a [G,M_max,K], sfa [G, K/128, align4(M_max)], b [G,N,K],
+    sfb [G, ceil(N/128), K/128], d [G,M_max,N], masked_m int32 [G]."""
+    _fp8(a, "a")
+    _fp8(b, "b")
+    G, M_max, K = a.shape
+    Gb, N, Kb_ = b.shape
+    if Gb != G or Kb_ != K:
+        raise ValueError("a and b disagree on G or K")
+    _f32(sfa, "sfa", (G, K // BLOCK, get_tma_aligned_size(M_max, 4)))
+    _f32(sfb, "sfb", (G, -(-N // BLOCK), K // BLOCK))
+    _out(d, (G, M_max, N))
+    _i32(masked_m, "masked_m", (G,))
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked(
+        _ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), _ptr(masked_m), G, M_max, N, K,
+        int(expected_m), _ptr(workspace), ws, _stream(stream)),
+        "dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked")

@@ -1,0 +1,581 @@
+// dg_api.cu -- host side of the C ABI declared in include/dg.h: argument checks, tile choice,
+// TMA tensor maps, and the launch of the sm_100a kernel on the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/dg.h"
+#include "dg_kernel.cuh"
+
+namespace {
+
+using dg::Params;
+
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
+constexpr int kMinDynSmem = 120 * 1024;  // keeps one CTA per SM (each takes all 512 TMEM columns)
+
+__device__ int g_device_error;  // the device error word read by dg_poll_device_error
+
+struct DeviceInfo {
+    bool init = false;
+    int status = DG_OK;
+    int num_sms = 0;
+    int smem_optin = 0;
+    int *err_ptr = nullptr;
+};
+
+std::mutex g_mutex;
+DeviceInfo g_dev[kMaxDevices];
+struct KernelSmem {
+    int static_bytes = -1;  // static shared memory of the kernel
+    int limit_set = 0;      // dynamic shared-memory limit already set on this device
+};
+KernelSmem g_smem[kMaxDevices][3][8];  // per device / layout / BN
+int g_num_sms_cap = 0;
+unsigned long long g_timeout_ns = kDefaultTimeoutNs;
+int g_override_bn = 0;
+int g_override_stages = 0;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+struct LastLaunch {
+    bool valid = false;
+    int block_n = 0, stages = 0, grid = 0, tiles = 0;
+};
+thread_local LastLaunch t_last;
+
+bool debug_enabled()
+{
+    static int v = -1;
+    if (v < 0) {
+        const char *e = std::getenv("DG_DEBUG");
+        v = (e && e[0] && e[0] != '0') ? 1 : 0;
+    }
+    return v == 1;
+}
+
+// Per-device set-up: checks for sm_100, reads SM count and shared-memory limit, and resolves
+// the address of the device error word.  Called with the device current.
+int device_setup(int &dev_out, DeviceInfo *&info)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return DG_ERR_UNSUPPORTED;
+    }
+    if (dev < 0 || dev >= kMaxDevices)
+        return DG_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.init) {
+        d.init = true;
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            d.status = DG_ERR_UNSUPPORTED;
+        } else if (major != 10 || minor != 0) {
+            d.status = DG_ERR_UNSUPPORTED;
+        } else {
+            cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+            cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) {
+                cudaGetLastError();
+                d.status = DG_ERR_CUDA;
+            } else {
+                d.err_ptr = static_cast<int *>(p);
+                d.status = DG_OK;
+            }
+        }
+        if (d.status == DG_OK && g_encode == nullptr) {
+            void *fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                    cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || fn == nullptr) {
+                cudaGetLastError();
+                d.status = DG_ERR_CUDA;
+            } else {
+                g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+            }
+        }
+    }
+    dev_out = dev;
+    info = &d;
+    return d.status;
+}
+
+bool aligned16(const void *p)
+{
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+int align4(int x)
+{
+    return (x + 3) / 4 * 4;
+}
+
+// 3-D tiled tensor map: dims/strides innermost first (strides in bytes for dims 1, 2).
+int make_map(CUtensorMap *map, CUtensorMapDataType dt, void *base, uint64_t d0, uint64_t d1,
+             uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1,
+             CUtensorMapSwizzle swz)
+{
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {stride1, stride2};
+    cuuint32_t box[3] = {b0, b1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, dt, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
+}
+
+template <int BN>
+constexpr int stage_bytes()
+{
+    return dg::Cfg<BN>::kStageBytes;
+}
+
+int stage_bytes_rt(int bn)
+{
+    return ((dg::kBlockM * dg::kBlockK + bn * dg::kBlockK + dg::kSfaBytes) + 1023) / 1024 * 1024;
+}
+
+using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, Params);
+
+template <int L, int BN>
+void *kernel_ptr()
+{
+    return reinterpret_cast<void *>(&dg::dg_gemm_kernel<L, BN>);
+}
+
+void *pick_kernel(int layout, int bn)
+{
+#define DG_CASE(BNV)                                                                           \
+    case BNV:                                                                                  \
+        return layout == dg::kDense        ? kernel_ptr<dg::kDense, BNV>()                       \
+               : layout == dg::kContiguous ? kernel_ptr<dg::kContiguous, BNV>()                  \
+                                           : kernel_ptr<dg::kMasked, BNV>();
+    switch (bn) {
+        DG_CASE(32)
+        DG_CASE(64)
+        DG_CASE(96)
+        DG_CASE(128)
+        DG_CASE(160)
+        DG_CASE(192)
+        DG_CASE(224)
+        DG_CASE(256)
+    default:
+        return nullptr;
+    }
+#undef DG_CASE
+}
+
+// Tile heuristic: among BN in {32..256} pick the one with the smallest estimated time, where a
+// tile of BN columns costs max(MMA time ~ BN, load time ~ 128 + BN) and tiles run in waves over
+// the SMs (non-power-of-two BN exists to even out the last wave).
+int choose_block_n(int rows_tiles, int N, int num_sms, long long expected_rows_total)
+{
+    (void)expected_rows_total;
+    int best_bn = 128;
+    double best = 1e300;
+    for (int bn = 32; bn <= 256; bn += 32) {
+        long long n_tiles = (N + bn - 1) / bn;
+        long long tiles = n_tiles * rows_tiles;
+        long long waves = (tiles + num_sms - 1) / num_sms;
+        double per_tile = std::max(static_cast<double>(bn), 0.55 * (128.0 + bn)) + 24.0;
+        double t = waves * per_tile;
+        // avoid wasting columns past N
+        double waste = static_cast<double>(n_tiles * bn - N) / N;
+        t *= 1.0 + 0.5 * waste;
+        if (t < best - 1e-9 || (std::abs(t - best) <= 1e-9 && bn > best_bn)) {
+            best = t;
+            best_bn = bn;
+        }
+    }
+    return best_bn;
+}
+
+struct LaunchArgs {
+    int layout;
+    const void *a;
+    const float *sfa;
+    const void *b;
+    const float *sfb;
+    void *d;
+    const int *m_indices;
+    const int *masked_m;
+    int M;  // dense M / M_total / M_max
+    int N, K, G;
+    int expected_m;
+    void *stream;
+};
+
+int launch(const LaunchArgs &args)
+{
+    int dev = 0;
+    DeviceInfo *info = nullptr;
+    int st = device_setup(dev, info);
+    if (st != DG_OK)
+        return st;
+
+    const int M = args.M, N = args.N, K = args.K, G = args.G;
+    const int num_kb = K / dg::kBlockK;
+    const int num_nb = (N + dg::kBlockK - 1) / dg::kBlockK;
+    const int m_tiles = (M + dg::kBlockM - 1) / dg::kBlockM;
+    int sms = info->num_sms;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (g_num_sms_cap > 0 && g_num_sms_cap < sms)
+            sms = g_num_sms_cap;
+    }
+
+    // tile choice
+    int bn;
+    int stages_override;
+    unsigned long long timeout;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        bn = g_override_bn;
+        stages_override = g_override_stages;
+        timeout = g_timeout_ns;
+    }
+    if (bn == 0) {
+        long long row_tiles = m_tiles;
+        if (args.layout == dg::kMasked) {
+            int em = args.expected_m > 0 ? std::min(args.expected_m, M) : M;
+            row_tiles = static_cast<long long>(G) * ((em + dg::kBlockM - 1) / dg::kBlockM);
+        }
+        bn = choose_block_n(static_cast<int>(std::max<long long>(1, row_tiles)), N, sms, 0);
+    }
+    const int n_tiles = (N + bn - 1) / bn;
+    const int sbytes = stage_bytes_rt(bn);
+    void *fn = pick_kernel(args.layout, bn);
+    if (fn == nullptr)
+        return DG_ERR_INVALID_ARG;
+    int dyn_smem = 0;
+    int stages = 0;
+    {
+        // The dynamic shared-memory limit of each kernel is raised once per device and only
+        // when a launch needs more, so launches can be captured into CUDA graphs.
+        std::lock_guard<std::mutex> lock(g_mutex);
+        KernelSmem &ks = g_smem[dev][args.layout][bn / 32 - 1];
+        if (ks.static_bytes < 0) {
+            cudaFuncAttributes fa;
+            cudaError_t e = cudaFuncGetAttributes(&fa, fn);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                if (debug_enabled())
+                    std::fprintf(stderr, "[dg] cudaFuncGetAttributes: %s\n", cudaGetErrorString(e));
+                return DG_ERR_CUDA;
+            }
+            ks.static_bytes = static_cast<int>(fa.sharedSizeBytes);
+        }
+        const int dyn_cap = info->smem_optin - ks.static_bytes;  // dynamic bytes allowed
+        stages = std::min(dg::kMaxStages, (dyn_cap - 1024) / sbytes);
+        if (stages_override > 0)
+            stages = std::min(stages, stages_override);
+        if (stages < 2)
+            return DG_ERR_UNSUPPORTED;
+        dyn_smem = stages * sbytes + 1024;  // + slack to align the stages to 1024 bytes
+        dyn_smem = std::min(std::max(dyn_smem, kMinDynSmem), dyn_cap);
+        if (ks.limit_set < dyn_smem) {
+            cudaError_t e =
+                cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                if (debug_enabled())
+                    std::fprintf(stderr, "[dg] cudaFuncSetAttribute(%d): %s\n", dyn_smem,
+                                 cudaGetErrorString(e));
+                return DG_ERR_CUDA;
+            }
+            ks.limit_set = dyn_smem;
+        }
+    }
+
+    // tensor maps
+    const int a_rows = (args.layout == dg::kMasked) ? M : M;
+    const int a_groups = (args.layout == dg::kMasked) ? G : 1;
+    const int b_groups = (args.layout == dg::kDense) ? 1 : G;
+    const int m4 = align4(M);
+    CUtensorMap map_a, map_b, map_sfa;
+    if (make_map(&map_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<void *>(args.a), K, a_rows,
+                 a_groups, static_cast<uint64_t>(K), static_cast<uint64_t>(K) * a_rows, dg::kBlockK,
+                 dg::kBlockM, CU_TENSOR_MAP_SWIZZLE_128B) != DG_OK ||
+        make_map(&map_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<void *>(args.b), K, N, b_groups,
+                 static_cast<uint64_t>(K), static_cast<uint64_t>(K) * N, dg::kBlockK, bn,
+                 CU_TENSOR_MAP_SWIZZLE_128B) != DG_OK ||
+        make_map(&map_sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float *>(args.sfa), m4,
+                 num_kb, a_groups, static_cast<uint64_t>(m4) * 4,
+                 static_cast<uint64_t>(m4) * 4 * num_kb, dg::kBlockM, 1,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) != DG_OK) {
+        if (debug_enabled())
+            std::fprintf(stderr, "[dg] cuTensorMapEncodeTiled failed\n");
+        return DG_ERR_CUDA;
+    }
+
+    Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.G = (args.layout == dg::kDense) ? 1 : G;
+    p.num_kb = num_kb;
+    p.num_nb = num_nb;
+    p.m_tiles = m_tiles;
+    p.n_tiles = n_tiles;
+    p.stages = stages;
+    p.raster_m = 16;
+    p.sfb = args.sfb;
+    p.d = static_cast<__nv_bfloat16 *>(args.d);
+    p.m_indices = args.m_indices;
+    p.masked_m = args.masked_m;
+    p.err = info->err_ptr;
+    p.timeout_ns = timeout;
+    long long tiles;
+    if (args.layout == dg::kMasked)
+        tiles = static_cast<long long>(G) * m_tiles * n_tiles;  // upper bound; exact on device
+    else
+        tiles = static_cast<long long>(m_tiles) * n_tiles;
+    if (tiles > 0x7FFFFFFFLL)
+        return DG_ERR_INVALID_ARG;
+    p.num_tiles = static_cast<int>(tiles);
+    int grid = static_cast<int>(std::min<long long>(sms, tiles));
+    if (grid <= 0)
+        return DG_OK;
+
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(dg::kNumThreads, 1, 1);
+    cfg.dynamicSmemBytes = dyn_smem;
+    cfg.stream = static_cast<cudaStream_t>(args.stream);
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
+    void *kargs[] = {&map_a, &map_b, &map_sfa, &p};
+    cudaError_t e = cudaLaunchKernelExC(&cfg, fn, kargs);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        if (debug_enabled())
+            std::fprintf(stderr, "[dg] launch failed: %s\n", cudaGetErrorString(e));
+        return DG_ERR_CUDA;
+    }
+    t_last.valid = true;
+    t_last.block_n = bn;
+    t_last.stages = stages;
+    t_last.grid = grid;
+    t_last.tiles = p.num_tiles;
+    if (debug_enabled())
+        std::fprintf(stderr, "[dg] layout=%d M=%d N=%d K=%d G=%d BN=%d stages=%d grid=%d tiles=%d smem=%d\n",
+                     args.layout, M, N, K, G, bn, stages, grid, p.num_tiles, dyn_smem);
+    return DG_OK;
+}
+
+int check_common(const void *a, const float *sfa, const void *b, const float *sfb, void *d, int N,
+                 int K)
+{
+    if (!a || !sfa || !b || !sfb || !d)
+        return DG_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(sfa) || !aligned16(b) || !aligned16(sfb) || !aligned16(d))
+        return DG_ERR_INVALID_ARG;
+    if (K <= 0 || K % dg::kBlockK != 0 || N <= 0 || N % 8 != 0)
+        return DG_ERR_INVALID_ARG;
+    return DG_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dg_gemm_fp8_fp8_bf16_nt(const void *a, const float *sfa, const void *b, const float *sfb,
+                            void *d, int M, int N, int K, void *workspace, size_t workspace_bytes,
+                            void *stream)
+{
+    (void)workspace;
+    (void)workspace_bytes;
+    if (M < 0)
+        return DG_ERR_INVALID_ARG;
+    if (M == 0)
+        return (N > 0 && N % 8 == 0 && K > 0 && K % dg::kBlockK == 0) ? DG_OK : DG_ERR_INVALID_ARG;
+    int st = check_common(a, sfa, b, sfb, d, N, K);
+    if (st != DG_OK)
+        return st;
+    LaunchArgs la{dg::kDense, a, sfa, b, sfb, d, nullptr, nullptr, M, N, K, 1, 0, stream};
+    return launch(la);
+}
+
+int dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(const void *a, const float *sfa, const void *b,
+                                                 const float *sfb, void *d, const int *m_indices,
+                                                 int M_total, int N, int K, int G, void *workspace,
+                                                 size_t workspace_bytes, void *stream)
+{
+    (void)workspace;
+    (void)workspace_bytes;
+    if (M_total < 0 || M_total % dg::kBlockM != 0 || G <= 0)
+        return DG_ERR_INVALID_ARG;
+    if (M_total == 0)
+        return (N > 0 && N % 8 == 0 && K > 0 && K % dg::kBlockK == 0) ? DG_OK : DG_ERR_INVALID_ARG;
+    int st = check_common(a, sfa, b, sfb, d, N, K);
+    if (st != DG_OK)
+        return st;
+    if (!m_indices || (reinterpret_cast<uintptr_t>(m_indices) & 3u))
+        return DG_ERR_INVALID_ARG;
+    LaunchArgs la{dg::kContiguous, a, sfa, b, sfb, d, m_indices, nullptr, M_total, N, K, G, 0,
+                  stream};
+    return launch(la);
+}
+
+int dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked(const void *a, const float *sfa, const void *b,
+                                             const float *sfb, void *d, const int *masked_m, int G,
+                                             int M_max, int N, int K, int expected_m,
+                                             void *workspace, size_t workspace_bytes, void *stream)
+{
+    (void)workspace;
+    (void)workspace_bytes;
+    if (G <= 0 || G > dg::kMaxMaskedGroups || M_max < 0 || expected_m < 0)
+        return DG_ERR_INVALID_ARG;
+    if (M_max == 0)
+        return (N > 0 && N % 8 == 0 && K > 0 && K % dg::kBlockK == 0) ? DG_OK : DG_ERR_INVALID_ARG;
+    int st = check_common(a, sfa, b, sfb, d, N, K);
+    if (st != DG_OK)
+        return st;
+    if (!masked_m || (reinterpret_cast<uintptr_t>(masked_m) & 3u))
+        return DG_ERR_INVALID_ARG;
+    LaunchArgs la{dg::kMasked, a, sfa, b, sfb, d, nullptr, masked_m, M_max, N, K, G, expected_m,
+                  stream};
+    return launch(la);
+}
+
+int dg_set_num_sms(int n)
+{
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int prev = g_num_sms_cap;
+    g_num_sms_cap = n > 0 ? n : 0;
+    return prev;
+}
+
+int dg_get_num_sms(void)
+{
+    int dev = 0;
+    DeviceInfo *info = nullptr;
+    int st = device_setup(dev, info);
+    if (st != DG_OK)
+        return st;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (g_num_sms_cap > 0 && g_num_sms_cap < info->num_sms)
+        return g_num_sms_cap;
+    return info->num_sms;
+}
+
+int dg_get_tma_aligned_size(int x, int elem_bytes)
+{
+    if (x < 0 || elem_bytes <= 0)
+        return DG_ERR_INVALID_ARG;
+    // smallest x' >= x with x' * elem_bytes % 16 == 0
+    long long step = 16;
+    long long g = elem_bytes;
+    long long a = step, b2 = g;
+    while (b2) {
+        long long tmp = a % b2;
+        a = b2;
+        b2 = tmp;
+    }
+    long long unit = step / a;  // elements per alignment unit
+    long long r = (static_cast<long long>(x) + unit - 1) / unit * unit;
+    return r > 0x7FFFFFFFLL ? DG_ERR_INVALID_ARG : static_cast<int>(r);
+}
+
+size_t dg_get_workspace_size(int kind, int M, int N, int K, int G)
+{
+    (void)kind;
+    (void)M;
+    (void)N;
+    (void)K;
+    (void)G;
+    return 0;
+}
+
+const char *dg_status_string(int status)
+{
+    switch (status) {
+    case DG_OK:
+        return "DG_OK";
+    case DG_ERR_INVALID_ARG:
+        return "DG_ERR_INVALID_ARG: invalid argument";
+    case DG_ERR_UNSUPPORTED:
+        return "DG_ERR_UNSUPPORTED: no sm_100 device or unsupported configuration";
+    case DG_ERR_CUDA:
+        return "DG_ERR_CUDA: a CUDA call failed";
+    case DG_ERR_TIMEOUT:
+        return "DG_ERR_TIMEOUT: a device pipeline wait timed out";
+    case DG_ERR_WORKSPACE:
+        return "DG_ERR_WORKSPACE: workspace missing or too small";
+    case DG_ERR_LAYOUT:
+        return "DG_ERR_LAYOUT: an index array broke its layout contract";
+    default:
+        return "unknown dg_status";
+    }
+}
+
+int dg_poll_device_error(void *stream)
+{
+    int dev = 0;
+    DeviceInfo *info = nullptr;
+    int st = device_setup(dev, info);
+    if (st != DG_OK)
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int value = 0;
+    const int zero = 0;
+    if (cudaMemcpyAsync(&value, info->err_ptr, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemcpyAsync(info->err_ptr, &zero, sizeof(int), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
+        cudaGetLastError();
+        return DG_ERR_CUDA;
+    }
+    return value;
+}
+
+unsigned long long dg_set_wait_timeout_ns(unsigned long long ns)
+{
+    std::lock_guard<std::mutex> lock(g_mutex);
+    unsigned long long prev = g_timeout_ns;
+    g_timeout_ns = ns ? ns : kDefaultTimeoutNs;
+    return prev;
+}
+
+int dg_set_config_override(int block_n, int num_stages)
+{
+    if (block_n != 0 && (block_n < 32 || block_n > 256 || block_n % 32 != 0))
+        return DG_ERR_INVALID_ARG;
+    if (num_stages != 0 && (num_stages < 2 || num_stages > dg::kMaxStages))
+        return DG_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    g_override_bn = block_n;
+    g_override_stages = num_stages;
+    return DG_OK;
+}
+
+int dg_get_last_launch(int *block_n, int *num_stages, int *grid, int *num_tiles)
+{
+    if (!t_last.valid)
+        return DG_ERR_INVALID_ARG;
+    if (block_n)
+        *block_n = t_last.block_n;
+    if (num_stages)
+        *num_stages = t_last.stages;
+    if (grid)
+        *grid = t_last.grid;
+    if (num_tiles)
+        *num_tiles = t_last.tiles;
+    return DG_OK;
+}
+
+}  // extern "C"

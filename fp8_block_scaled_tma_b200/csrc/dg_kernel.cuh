@@ -1,0 +1,536 @@
+// dg_kernel.cuh -- the sm_100a FP8 block-scaled NT GEMM kernel (dense, contiguous-grouped and
+// masked-grouped layouts share it; only the tile scheduler differs).
+//
+// Method (DeepSeek開源第三彈 -- the DeepGEMM release write-up -- "深入了解DeepGEMM"): FP8 inputs
+// with DeepSeek-V3 fine-grained scales (fp32 per 1x128 tile of A, per 128x128 block of B), and
+// two-level accumulation: the tensor cores form the product of one 128-wide K slice, the CUDA
+// cores multiply it by sa*sb and add it to an fp32 accumulator.  The layouts are those of
+// "如何使用" (NT dense, MoE contiguous, MoE masked).
+//
+// Blackwell design (one CTA of 384 threads per SM, persistent over output tiles):
+//   warp 0          TMA producer: per K block loads A [128 x 128 B], B [BN x 128 B] (both with
+//                   the 128-byte swizzle) and the 128 fp32 scales of A into one pipeline stage.
+//   warp 1          allocates tensor memory, then issues 4 x tcgen05.mma kind::f8f6f4 (K = 32
+//                   each) per K block into one of NB TMEM buffers of BN fp32 columns, and
+//                   commits the stage (free) and the buffer (full) to mbarriers.
+//   warps 4..11     promotion: each thread owns one output row (its TMEM lane) and BN/2
+//                   columns; per K block it loads the fresh partial from TMEM, frees the
+//                   buffer, and adds partial * sa[row] * sb[block] into fp32 registers.  After
+//                   the last K block it rounds to bf16 and stores its row segment.
+// Every wait is bounded by a %globaltimer limit; on expiry the kernel records DG_ERR_TIMEOUT,
+// drains its outstanding copies and MMAs, frees tensor memory and returns.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "dg_ptx.cuh"
+
+namespace dg {
+
+constexpr int kBlockM = 128;           // rows per tile (one TMEM lane each)
+constexpr int kBlockK = 128;           // K per scale block = K per promotion
+constexpr int kUmmaK = 32;             // K of one tcgen05.mma kind::f8f6f4
+constexpr int kNumThreads = 384;
+constexpr int kNumMathWarps = 8;
+constexpr int kFirstMathWarp = 4;
+constexpr int kMaxStages = 8;
+constexpr int kTmemCols = 512;
+constexpr int kMaxMaskedGroups = 1024;
+constexpr int kSfaBytes = kBlockM * 4;
+constexpr uint64_t kDrainTimeoutNs = 1000000000ull;  // fixed bound for the wind-down waits
+
+constexpr int kErrTimeout = -4;
+constexpr int kErrLayout = -6;
+
+enum Layout : int { kDense = 0, kContiguous = 1, kMasked = 2 };
+
+struct Params {
+    int M;          // dense: M, contiguous: M_total, masked: M_max
+    int N;
+    int K;
+    int G;
+    int num_kb;     // K / 128
+    int num_nb;     // ceil(N / 128): scale blocks of B along N
+    int m_tiles;    // ceil(M / 128)
+    int n_tiles;    // ceil(N / BN)
+    int num_tiles;  // dense / contiguous: m_tiles * n_tiles; masked: computed on the device
+    int stages;
+    int raster_m;   // m-tiles per raster band (dense / contiguous)
+    const float *sfb;
+    __nv_bfloat16 *d;
+    const int *m_indices;
+    const int *masked_m;
+    int *err;
+    unsigned long long timeout_ns;
+};
+
+template <int BN>
+struct Cfg {
+    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN must be a multiple of 32 in [32, 256]");
+    static constexpr int kCols = BN / 2;                      // columns per promotion thread
+    static constexpr int kChunk = (kCols % 32 == 0) ? 32 : 16;
+    static constexpr int kNumChunks = kCols / kChunk;
+    static constexpr int kTmemBufs = (kTmemCols / BN) >= 4 ? 4 : (kTmemCols / BN);
+    static constexpr int kABytes = kBlockM * kBlockK;         // 16 KB
+    static constexpr int kBBytes = BN * kBlockK;
+    static constexpr int kStageBytes = ((kABytes + kBBytes + kSfaBytes) + 1023) / 1024 * 1024;
+    static constexpr uint32_t kTxBytes = kABytes + kBBytes + kSfaBytes;
+    static constexpr uint32_t kIdesc = ptx::idesc_e4m3_f32(kBlockM, BN);
+};
+
+// Static shared memory: barriers and the bookkeeping words.
+struct SmemCtl {
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
+    uint64_t tmem_full[4];
+    uint64_t tmem_empty[4];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int total_tiles;
+    int tile_prefix[kMaxMaskedGroups + 1];
+};
+
+struct Tile {
+    int g;       // group (expert) of the tile; 0 for dense
+    int m0;      // first row of the tile within its group
+    int n0;      // first column
+    int a_z;     // TMA z coordinate of A / SFA (group for masked, else 0)
+};
+
+__device__ __forceinline__ void record_error(int *err, int code)
+{
+    atomicCAS(err, 0, code);
+}
+
+// Resolves tile t to its coordinates.  Returns false when the tile has no valid row and must
+// be skipped (contiguous layout only).  All roles call it with the same t and read the same
+// (read-only) index arrays, so they agree.
+template <int L>
+__device__ __forceinline__ bool resolve_tile(const Params &p, const SmemCtl &ctl, int t, Tile &ti)
+{
+    if (L == kMasked) {
+        // find g with prefix[g] <= t < prefix[g + 1]
+        int lo = 0, hi = p.G - 1;
+        while (lo < hi) {
+            int mid = (lo + hi + 1) >> 1;
+            if (ctl.tile_prefix[mid] <= t)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        int g = lo;
+        int mm = __ldg(p.masked_m + g);
+        mm = mm < 0 ? 0 : (mm > p.M ? p.M : mm);
+        int mt = (mm + kBlockM - 1) / kBlockM;
+        int local = t - ctl.tile_prefix[g];
+        ti.g = g;
+        ti.m0 = (local % mt) * kBlockM;
+        ti.n0 = (local / mt);  // scaled by BN by the caller
+        ti.a_z = g;
+        return true;
+    } else {
+        int band = p.raster_m * p.n_tiles;
+        int b = t / band;
+        int r = t - b * band;
+        int m_base = b * p.raster_m;
+        int h = p.m_tiles - m_base;
+        h = h < p.raster_m ? h : p.raster_m;
+        ti.m0 = (m_base + r % h) * kBlockM;
+        ti.n0 = r / h;
+        ti.a_z = 0;
+        ti.g = 0;
+        if (L == kContiguous) {
+            int g = __ldg(p.m_indices + ti.m0);
+            if (g < 0) {
+                int end = ti.m0 + kBlockM < p.M ? ti.m0 + kBlockM : p.M;
+                for (int r2 = ti.m0 + 1; r2 < end && g < 0; ++r2)
+                    g = __ldg(p.m_indices + r2);
+            }
+            if (g < 0)
+                return false;          // an all-padding tile: nothing to write
+            if (g >= p.G) {
+                record_error(p.err, kErrLayout);
+                return false;
+            }
+            ti.g = g;
+        }
+        return true;
+    }
+}
+
+// Bounded wait by one thread.  Returns false on timeout or when another role aborted.
+__device__ __forceinline__ bool wait_one(uint32_t bar, uint32_t parity, const Params &p,
+                                         volatile int *abort_flag)
+{
+    if (ptx::mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = ptx::global_timer_ns();
+    while (true) {
+        if (ptx::mbar_try_wait(bar, parity))
+            return true;
+        if (*abort_flag)
+            return false;
+        if (ptx::global_timer_ns() - t0 > p.timeout_ns) {
+            *abort_flag = 1;
+            record_error(p.err, kErrTimeout);
+            return false;
+        }
+    }
+}
+
+// Wait used while winding down: a fixed bound independent of the configurable limit.
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity)
+{
+    const uint64_t t0 = ptx::global_timer_ns();
+    while (!ptx::mbar_try_wait(bar, parity)) {
+        if (ptx::global_timer_ns() - t0 > kDrainTimeoutNs)
+            return false;
+    }
+    return true;
+}
+
+template <int L, int BN>
+__global__ void __launch_bounds__(kNumThreads, 1)
+    dg_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                   const __grid_constant__ CUtensorMap tmap_b,
+                   const __grid_constant__ CUtensorMap tmap_sfa, const Params p)
+{
+    using C = Cfg<BN>;
+    __shared__ SmemCtl ctl;
+    extern __shared__ uint8_t smem_raw[];
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    // stage buffers start on a 1024-byte boundary (the 128-byte swizzle atom)
+    const uint32_t smem_base = (ptx::smem_addr(smem_raw) + 1023u) & ~1023u;
+    uint8_t *smem_gen = smem_raw + (smem_base - ptx::smem_addr(smem_raw));
+
+    auto stage_a = [&](int s) { return smem_base + s * C::kStageBytes; };
+    auto stage_b = [&](int s) { return smem_base + s * C::kStageBytes + C::kABytes; };
+    auto stage_sfa = [&](int s) {
+        return reinterpret_cast<const float *>(smem_gen + s * C::kStageBytes + C::kABytes +
+                                               C::kBBytes);
+    };
+    const uint32_t bar_full = ptx::smem_addr(&ctl.full[0]);
+    const uint32_t bar_empty = ptx::smem_addr(&ctl.empty[0]);
+    const uint32_t bar_tfull = ptx::smem_addr(&ctl.tmem_full[0]);
+    const uint32_t bar_tempty = ptx::smem_addr(&ctl.tmem_empty[0]);
+    const uint32_t bar_drain = ptx::smem_addr(&ctl.drain);
+    volatile int *abort_flag = &ctl.abort_flag;
+
+    // ---- set-up ------------------------------------------------------------------------
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            ptx::mbar_init(bar_full + 8 * s, 1);
+            ptx::mbar_init(bar_empty + 8 * s, 1 + kNumMathWarps);
+        }
+        for (int b = 0; b < C::kTmemBufs; ++b) {
+            ptx::mbar_init(bar_tfull + 8 * b, 1);
+            ptx::mbar_init(bar_tempty + 8 * b, kNumMathWarps);
+        }
+        ptx::mbar_init(bar_drain, 1);
+        ctl.abort_flag = 0;
+        ptx::fence_mbar_init();
+        ptx::prefetch_tmap(&tmap_a);
+        ptx::prefetch_tmap(&tmap_b);
+        ptx::prefetch_tmap(&tmap_sfa);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(ptx::smem_addr(&ctl.tmem_base), kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    if (L == kMasked) {
+        if (warp == 2 && lane == 0) {
+            // prefix over groups of (m-tiles of the group) * n_tiles
+            int acc = 0;
+            for (int g = 0; g < p.G; ++g) {
+                ctl.tile_prefix[g] = acc;
+                int mm = __ldg(p.masked_m + g);
+                if (mm < 0 || mm > p.M) {
+                    if (blockIdx.x == 0)
+                        record_error(p.err, kErrLayout);
+                    mm = mm < 0 ? 0 : p.M;
+                }
+                acc += (mm + kBlockM - 1) / kBlockM * p.n_tiles;
+            }
+            ctl.tile_prefix[p.G] = acc;
+            ctl.total_tiles = acc;
+        }
+    } else if (threadIdx.x == 0) {
+        ctl.total_tiles = p.num_tiles;
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = ctl.tmem_base;
+    const int num_tiles = ctl.total_tiles;
+
+    if (warp < kFirstMathWarp) {
+        ptx::setmaxnreg_dec<40>();
+        if (warp == 0 && lane == 0) {
+            // ---------------- TMA producer ----------------
+            uint32_t it = 0;
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                Tile ti;
+                if (!resolve_tile<L>(p, ctl, t, ti))
+                    continue;
+                const int n0 = ti.n0 * BN;
+                const int a_y = ti.m0;
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!wait_one(bar_empty + 8 * s, ph ^ 1, p, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = bar_full + 8 * s;
+                    ptx::mbar_arrive_expect_tx(fb, C::kTxBytes);
+                    ptx::tma_load_3d(stage_a(s), &tmap_a, fb, kb * kBlockK, a_y, ti.a_z);
+                    ptx::tma_load_3d(stage_b(s), &tmap_b, fb, kb * kBlockK, n0, ti.g);
+                    ptx::tma_load_3d(ptx::smem_addr(stage_sfa(s)), &tmap_sfa, fb, ti.m0, kb,
+                                     ti.a_z);
+                    ++it;
+                    if (++s == p.stages) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+            }
+            // Wind down: every issued load must have landed before the CTA may exit.  The
+            // last min(it, stages) loads are the only ones that can still be in flight.
+            int pending = it < static_cast<uint32_t>(p.stages) ? static_cast<int>(it) : p.stages;
+            int ds = s;
+            uint32_t dph = ph;
+            for (int i = 0; i < pending; ++i) {
+                if (--ds < 0) {
+                    ds = p.stages - 1;
+                    dph ^= 1;
+                }
+                wait_drain(bar_full + 8 * ds, dph);
+            }
+        } else if (warp == 1 && lane == 0) {
+            // ---------------- MMA issuer ----------------
+            int s = 0;
+            uint32_t ph = 0;
+            int buf = 0;
+            uint32_t bph = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                Tile ti;
+                if (!resolve_tile<L>(p, ctl, t, ti))
+                    continue;
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!wait_one(bar_tempty + 8 * buf, bph ^ 1, p, abort_flag) ||
+                        !wait_one(bar_full + 8 * s, ph, p, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint64_t adesc = ptx::sdesc_kmajor_sw128(stage_a(s));
+                    const uint64_t bdesc = ptx::sdesc_kmajor_sw128(stage_b(s));
+                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+#pragma unroll
+                    for (int k = 0; k < kBlockK / kUmmaK; ++k) {
+                        // advance the start address by 32 bytes (2 x 16 B) per K step
+                        ptx::mma_f8f6f4(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::kIdesc,
+                                        k > 0 ? 1u : 0u);
+                    }
+                    ptx::mma_commit(bar_empty + 8 * s);
+                    ptx::mma_commit(bar_tfull + 8 * buf);
+                    if (++s == p.stages) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                    if (++buf == C::kTmemBufs) {
+                        buf = 0;
+                        bph ^= 1;
+                    }
+                }
+            }
+            // Wind down: all issued MMAs complete before tensor memory is released.
+            ptx::mma_commit(bar_drain);
+            wait_drain(bar_drain, 0);
+        }
+    } else {
+        ptx::setmaxnreg_inc<232>();
+        // ---------------- promotion + epilogue ----------------
+        const int mw = warp - kFirstMathWarp;     // 0..7
+        const int half = mw / 4;                  // which half of the BN columns
+        const int q = warp % 4;                   // TMEM lane quarter this warp may access
+        const int row = q * 32 + lane;            // row within the tile
+        const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>(half * C::kCols);
+        int s = 0;
+        uint32_t ph = 0;
+        int buf = 0;
+        uint32_t bph = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            Tile ti;
+            if (!resolve_tile<L>(p, ctl, t, ti))
+                continue;
+            const int n0 = ti.n0 * BN;
+            const int col0 = n0 + half * C::kCols;  // first global column of this thread
+            // the (at most two) 128-column scale blocks of B this thread's columns touch
+            const int nb_lo = min(col0 / kBlockK, p.num_nb - 1);
+            const int nb_hi = min((col0 + C::kCols - 1) / kBlockK, p.num_nb - 1);
+            uint32_t hi_mask = 0;
+#pragma unroll
+            for (int j = 0; j < C::kCols / 16; ++j)
+                if ((col0 + 16 * j) / kBlockK > nb_lo)
+                    hi_mask |= 1u << j;
+            const float *sfb_lo = p.sfb + (static_cast<size_t>(ti.g) * p.num_nb + nb_lo) * p.num_kb;
+            const float *sfb_hi = p.sfb + (static_cast<size_t>(ti.g) * p.num_nb + nb_hi) * p.num_kb;
+
+            float acc[C::kCols];
+#pragma unroll
+            for (int j = 0; j < C::kCols; ++j)
+                acc[j] = 0.0f;
+
+            for (int kb = 0; kb < p.num_kb; ++kb) {
+                const float sb_lo = __ldg(sfb_lo + kb);
+                const float sb_hi = __ldg(sfb_hi + kb);
+                bool w = wait_one(bar_full + 8 * s, ph, p, abort_flag) &&
+                         wait_one(bar_tfull + 8 * buf, bph, p, abort_flag);
+                w = __all_sync(0xffffffffu, w);
+                if (!w) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const float sa = stage_sfa(s)[row];
+                const float scale_lo = sa * sb_lo;
+                const float scale_hi = sa * sb_hi;
+                const uint32_t taddr = lane_base + static_cast<uint32_t>(buf * BN);
+
+                uint32_t r0[16], r1[16];
+                if (C::kChunk == 32) {
+                    uint32_t r2[16], r3[16];
+                    ptx::tmem_ld_x16(taddr, r0);
+                    ptx::tmem_ld_x16(taddr + 16, r1);
+                    ptx::tmem_wait_ld(r0);
+                    ptx::tmem_wait_ld(r1);
+#pragma unroll
+                    for (int c = 0; c < C::kNumChunks; ++c) {
+                        if (c + 1 < C::kNumChunks) {
+                            ptx::tmem_ld_x16(taddr + 32 * (c + 1), r2);
+                            ptx::tmem_ld_x16(taddr + 32 * (c + 1) + 16, r3);
+                        } else {
+                            // all partials of this K block are in registers: free the buffer
+                            ptx::tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) {
+                                ptx::mbar_arrive(bar_tempty + 8 * buf);
+                                ptx::mbar_arrive(bar_empty + 8 * s);
+                            }
+                        }
+                        const float sc0 = ((hi_mask >> (2 * c)) & 1u) ? scale_hi : scale_lo;
+                        const float sc1 = ((hi_mask >> (2 * c + 1)) & 1u) ? scale_hi : scale_lo;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            acc[32 * c + j] = fmaf(__uint_as_float(r0[j]), sc0, acc[32 * c + j]);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            acc[32 * c + 16 + j] =
+                                fmaf(__uint_as_float(r1[j]), sc1, acc[32 * c + 16 + j]);
+                        if (c + 1 < C::kNumChunks) {
+                            ptx::tmem_wait_ld(r2);
+                            ptx::tmem_wait_ld(r3);
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                r0[j] = r2[j];
+                                r1[j] = r3[j];
+                            }
+                        }
+                    }
+                } else {
+                    ptx::tmem_ld_x16(taddr, r0);
+                    ptx::tmem_wait_ld(r0);
+#pragma unroll
+                    for (int c = 0; c < C::kNumChunks; ++c) {
+                        if (c + 1 < C::kNumChunks) {
+                            ptx::tmem_ld_x16(taddr + 16 * (c + 1), r1);
+                        } else {
+                            ptx::tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) {
+                                ptx::mbar_arrive(bar_tempty + 8 * buf);
+                                ptx::mbar_arrive(bar_empty + 8 * s);
+                            }
+                        }
+                        const float sc = ((hi_mask >> c) & 1u) ? scale_hi : scale_lo;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            acc[16 * c + j] = fmaf(__uint_as_float(r0[j]), sc, acc[16 * c + j]);
+                        if (c + 1 < C::kNumChunks) {
+                            ptx::tmem_wait_ld(r1);
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                r0[j] = r1[j];
+                        }
+                    }
+                }
+                if (++s == p.stages) {
+                    s = 0;
+                    ph ^= 1;
+                }
+                if (++buf == C::kTmemBufs) {
+                    buf = 0;
+                    bph ^= 1;
+                }
+            }
+            if (!ok)
+                break;
+
+            // ---- epilogue: bf16 rounding and row-predicated stores ----
+            const int grow = ti.m0 + row;  // row within the group
+            bool valid;
+            size_t out_row;
+            if (L == kDense) {
+                valid = grow < p.M;
+                out_row = static_cast<size_t>(grow);
+            } else if (L == kContiguous) {
+                valid = false;
+                if (grow < p.M) {
+                    const int gi = __ldg(p.m_indices + grow);
+                    valid = gi == ti.g;
+                    if (gi >= 0 && gi != ti.g)
+                        record_error(p.err, kErrLayout);
+                }
+                out_row = static_cast<size_t>(grow);
+            } else {
+                int mm = __ldg(p.masked_m + ti.g);
+                mm = mm < 0 ? 0 : (mm > p.M ? p.M : mm);
+                valid = grow < mm;
+                out_row = static_cast<size_t>(ti.g) * p.M + grow;
+            }
+            if (valid) {
+                __nv_bfloat16 *drow = p.d + out_row * p.N;
+#pragma unroll
+                for (int j = 0; j < C::kCols / 8; ++j) {
+                    const int col = col0 + 8 * j;
+                    if (col < p.N) {
+                        ptx::st_global_v4(drow + col, ptx::pack_bf16x2(acc[8 * j], acc[8 * j + 1]),
+                                          ptx::pack_bf16x2(acc[8 * j + 2], acc[8 * j + 3]),
+                                          ptx::pack_bf16x2(acc[8 * j + 4], acc[8 * j + 5]),
+                                          ptx::pack_bf16x2(acc[8 * j + 6], acc[8 * j + 7]));
+                    }
+                }
+            }
+        }
+    }
+
+    // ---- tear-down: everyone is past its last tcgen05 operation ----------------------------
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+}  // namespace dg

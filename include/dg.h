@@ -1,0 +1,143 @@
+/*
+ * dg.h -- C ABI of the B200 (sm_100a) FP8 block-scaled NT GEMM library.
+ *
+ * The operation (DeepSeek開源第三彈 -- the DeepGEMM release write-up -- sections
+ * "深入了解DeepGEMM" and "如何使用"): an FP8 GEMM with fine-grained scaling taken from DeepSeek-V3,
+ * in the NT layout (non-transposed left operand, transposed right operand), with bf16 output:
+ *
+ *     D[m][n] = sum_kb  sfa(m, kb) * sfb(n / 128, kb) * sum_{k in K-block kb} a[m][k] * b[n][k]
+ *
+ * a and b hold e4m3 codes (OCP FP8 E4M3, no infinities, max 448).  sfa is the fp32 scale of
+ * each 1x128 tile of a (one per row and 128-wide K block), sfb the fp32 scale of each 128x128
+ * block of b.  The product of each 128-wide K slice is formed on the tensor cores and then
+ * scaled and added into an fp32 accumulator on the CUDA cores (the "two-level accumulation"
+ * of "深入了解DeepGEMM"), then rounded to bf16 (round to nearest even).
+ *
+ * Conventions for every call below:
+ *   - Every pointer is a DEVICE pointer owned by the caller.  The library never allocates,
+ *     frees or synchronises on these calls; all work is enqueued on `stream`
+ *     (a cudaStream_t passed as void*; NULL means the legacy default stream).
+ *   - Base pointers must be 16-byte aligned.  K must be a positive multiple of 128 and N a
+ *     positive multiple of 8 (16-byte output rows).
+ *   - Return value: DG_OK (0) when the work was enqueued, otherwise a negative dg_status.
+ *     Errors found before the launch (DG_ERR_INVALID_ARG, DG_ERR_UNSUPPORTED) launch
+ *     nothing and leave d untouched.  DG_ERR_CUDA reports a failed launch.
+ *   - Scales of a are stored MN-major ("TMA-aligned", see dg_get_tma_aligned_size): for each
+ *     K block kb, the scales of all rows are contiguous, padded to a multiple of 4 rows:
+ *       sfa[kb * align4(M) + m].
+ *     Scales of b are row-major per 128-row block: sfb[nb * (K/128) + kb].
+ *   - Device-side contract checks and the pipeline watchdog record an error word that
+ *     dg_poll_device_error() reads (see there); they never trap.
+ */
+#ifndef DG_B200_DG_H
+#define DG_B200_DG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dg_status {
+    DG_OK = 0,
+    DG_ERR_INVALID_ARG = -1, /* null/misaligned pointer, bad size, K % 128 != 0, N % 8 != 0 */
+    DG_ERR_UNSUPPORTED = -2, /* no CUDA device, or the current device is not sm_100 */
+    DG_ERR_CUDA = -3,        /* a CUDA runtime/driver call failed (launch, tensor map) */
+    DG_ERR_TIMEOUT = -4,     /* device: a pipeline wait exceeded its time limit */
+    DG_ERR_WORKSPACE = -5,   /* workspace missing or smaller than dg_get_workspace_size() */
+    DG_ERR_LAYOUT = -6       /* device: an index array broke its contract (see each call) */
+} dg_status;
+
+/* Dense GEMM, "gemm_fp8_fp8_bf16_nt" of "如何使用".
+ *   a   e4m3 [M][K] row-major          sfa fp32 [K/128][align4(M)]  (MN-major)
+ *   b   e4m3 [N][K] row-major          sfb fp32 [ceil(N/128)][K/128]
+ *   d   bf16 [M][N] row-major (written: all M x N elements)
+ * M >= 0 (M == 0 is a no-op).  workspace / workspace_bytes: pass NULL / 0 unless
+ * dg_get_workspace_size(0, M, N, K, 1) > 0. */
+int dg_gemm_fp8_fp8_bf16_nt(const void *a, const float *sfa, const void *b, const float *sfb,
+                            void *d, int M, int N, int K, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/* Contiguous-layout grouped GEMM for MoE, "m_grouped_gemm_fp8_fp8_bf16_nt_contiguous" of
+ * "如何使用" (the token rows of several experts are concatenated along M).
+ *   a          e4m3 [M_total][K]          sfa fp32 [K/128][M_total]
+ *   b          e4m3 [G][N][K]             sfb fp32 [G][ceil(N/128)][K/128]
+ *   d          bf16 [M_total][N]
+ *   m_indices  int32 [M_total] on the device: the expert of each row, in [0, G), or -1 for a
+ *              padding row.  Rows with -1 are NOT written.
+ * M_total must be a multiple of 128 and every aligned 128-row tile may hold rows of one
+ * expert only (plus -1 rows): the segments of each expert are padded to 128 rows.  A tile
+ * that breaks this, or an index outside [-1, G), sets DG_ERR_LAYOUT on the device and the
+ * offending rows are not written. */
+int dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(const void *a, const float *sfa, const void *b,
+                                                 const float *sfb, void *d, const int *m_indices,
+                                                 int M_total, int N, int K, int G,
+                                                 void *workspace, size_t workspace_bytes,
+                                                 void *stream);
+
+/* Masked-layout grouped GEMM for MoE decoding, "m_grouped_gemm_fp8_fp8_bf16_nt_masked" of
+ * "如何使用" (a fixed-size batch per expert of which only the first masked_m[g] rows hold
+ * tokens).
+ *   a          e4m3 [G][M_max][K]         sfa fp32 [G][K/128][align4(M_max)]
+ *   b          e4m3 [G][N][K]             sfb fp32 [G][ceil(N/128)][K/128]
+ *   d          bf16 [G][M_max][N]
+ *   masked_m   int32 [G] on the device, 0 <= masked_m[g] <= M_max.  Rows r >= masked_m[g] of
+ *              group g are NOT written.  A value outside [0, M_max] sets DG_ERR_LAYOUT and is
+ *              clamped.
+ *   expected_m host-side hint of the typical masked_m (used only to choose tiles; never
+ *              changes results).  masked_m is read on the device only, so the call needs no
+ *              host synchronisation. */
+int dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked(const void *a, const float *sfa, const void *b,
+                                             const float *sfb, void *d, const int *masked_m,
+                                             int G, int M_max, int N, int K, int expected_m,
+                                             void *workspace, size_t workspace_bytes,
+                                             void *stream);
+
+/* The SM-count utility of "如何使用": caps the number of SMs the persistent kernels occupy so
+ * that other work (for example communication kernels) can run beside them.  n <= 0 restores
+ * "all SMs".  Returns the previous cap (0 = all). */
+int dg_set_num_sms(int n);
+
+/* Number of SMs the kernels will use on the current device (the cap, or all SMs).  Returns
+ * DG_ERR_UNSUPPORTED when no device is present. */
+int dg_get_num_sms(void);
+
+/* The TMA-alignment utility of "如何使用": the smallest x' >= x such that x' * elem_bytes is a
+ * multiple of 16 bytes (the tensor-memory-accelerator stride rule).  For the fp32 scales of
+ * a this is align4(M).  Returns DG_ERR_INVALID_ARG for x < 0 or elem_bytes <= 0. */
+int dg_get_tma_aligned_size(int x, int elem_bytes);
+
+/* Bytes of workspace a call of `kind` (0 dense, 1 contiguous, 2 masked) with these sizes
+ * needs.  0 means workspace may be NULL. */
+size_t dg_get_workspace_size(int kind, int M, int N, int K, int G);
+
+/* Static, human-readable text for a dg_status value. */
+const char *dg_status_string(int status);
+
+/* Reads the device error word that contract checks and the pipeline watchdog set, resets it
+ * to 0, and returns it (DG_OK, DG_ERR_TIMEOUT or DG_ERR_LAYOUT).  This call SYNCHRONISES
+ * `stream`; it is meant for tests and debugging, not for the hot path. */
+int dg_poll_device_error(void *stream);
+
+/* Time limit, in nanoseconds, of every pipeline wait inside the kernels (default 2e9).
+ * A wait that exceeds it sets DG_ERR_TIMEOUT on the device and the kernel winds down
+ * (outstanding copies and tensor-core work are drained, tensor memory is freed) instead of
+ * hanging.  0 restores the default.  Returns the previous value. */
+unsigned long long dg_set_wait_timeout_ns(unsigned long long ns);
+
+/* Tuning/testing override of the tile choice: block_n in {32, 64, ..., 256} (the N extent of a
+ * tile; 0 = heuristic) and the number of shared-memory pipeline stages (0 = as many as fit).
+ * Returns DG_ERR_INVALID_ARG for unsupported values. */
+int dg_set_config_override(int block_n, int num_stages);
+
+/* Describes the most recent launch on this host thread: fills any non-NULL pointer with the
+ * chosen block_n, pipeline stages, grid size (CTAs) and tile count.  Returns DG_OK, or
+ * DG_ERR_INVALID_ARG when nothing was launched yet. */
+int dg_get_last_launch(int *block_n, int *num_stages, int *grid, int *num_tiles);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DG_B200_DG_H */

@@ -1,0 +1,120 @@
+"""Parity helpers shared by the GPU tests: moving seeded inputs to the device, running the
+library, and comparing with the oracle under the stated tolerance.
+
+Tolerance (per element, on valid rows):  |D - Dref| <= 2 * ulp_bf16(Dref) + 1e-3 * sum_k |sa a| |sb b|
+with ulp_bf16(x) = 2^(max(floor(log2 |x|), -126) - 7) (2^-133 for x = 0); and per matrix
+1 - 2<D,Dref> / (<D,D> + <Dref,Dref>) <= 1e-5 in fp64.  Rows the call must not write keep the
+sentinel bit pattern exactly.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+SENTINEL = 0xFFFF  # a bf16 NaN pattern no finite result can take
+ULP_FACTOR = 2.0
+MAG_FACTOR = 1e-3
+DIFF_MAX = 1e-5
+
+
+def bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def ulp_bf16(x: np.ndarray) -> np.ndarray:
+    ax = np.abs(x)
+    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    e = np.where(ax > 0, np.maximum(e, -126), -126)
+    return np.exp2(e - 7)
+
+
+def compare(got_bits: np.ndarray, ref_bits: np.ndarray, mag: np.ndarray, acc=None) -> dict:
+    """Element and matrix checks over matching arrays of valid entries.  With ``acc`` (the
+    oracle's fp64 value before rounding) it also reports the error beyond one bf16 rounding:
+    excess = max(0, |D - acc| - ulp_bf16(acc)) / mag, which fp32 accumulation keeps near 1e-6."""
+    got = bits_to_f64(got_bits)
+    ref = bits_to_f64(ref_bits)
+    assert np.all(np.isfinite(ref)), "oracle produced a non-finite value"
+    err = np.abs(got - ref)
+    bound = ULP_FACTOR * ulp_bf16(ref) + MAG_FACTOR * mag
+    bad = ~(err <= bound)
+    den = float(np.sum(got * got) + np.sum(ref * ref))
+    diff = 0.0 if den == 0 else 1.0 - 2.0 * float(np.sum(got * ref)) / den
+    excess = 0.0
+    if acc is not None and err.size:
+        acc = np.asarray(acc, dtype=np.float64)
+        ex = np.maximum(0.0, np.abs(got - acc) - ulp_bf16(acc)) / np.maximum(mag, 1e-300)
+        excess = float(np.max(ex))
+    return dict(n_bad=int(bad.sum()), n=int(err.size), diff=diff, excess=excess,
+                first_bad=None if not bad.any() else tuple(int(i) for i in np.argwhere(bad)[0]))
+
+
+def assert_close(got_bits, ref_bits, mag, what: str = "", acc=None) -> dict:
+    r = compare(got_bits, ref_bits, mag, acc)
+    assert r["n_bad"] == 0, f"{what}: {r['n_bad']}/{r['n']} elements out of tolerance, first at {r['first_bad']}: {r}"
+    assert r["diff"] <= DIFF_MAX, f"{what}: matrix diff {r['diff']} > {DIFF_MAX}"
+    return r
+
+
+def to_dev_u8(x: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def to_dev_f32(x: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda()
+
+
+def sentinel_out(shape) -> torch.Tensor:
+    # int16 -1 is the bit pattern 0xFFFF (SENTINEL)
+    return torch.full(shape, -1, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+
+
+def out_bits(d: torch.Tensor) -> np.ndarray:
+    return d.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def run_dense(dg, case, d=None) -> torch.Tensor:
+    a = to_dev_u8(case.a)
+    b = to_dev_u8(case.b)
+    sfa = dg.sfa_mn_major(to_dev_f32(case.sa))
+    sfb = to_dev_f32(case.sb)
+    if d is None:
+        d = sentinel_out((case.M, case.N))
+    dg.dg_gemm_fp8_fp8_bf16_nt(a, sfa, b, sfb, d)
+    torch.cuda.synchronize()
+    return d
+
+
+def run_contiguous(dg, case, a=None, sa=None) -> torch.Tensor:
+    a = to_dev_u8(case.a if a is None else a)
+    sfa = dg.sfa_mn_major(to_dev_f32(case.sa if sa is None else sa))
+    b = to_dev_u8(case.b)
+    sfb = to_dev_f32(case.sb)
+    mi = torch.from_numpy(case.m_indices).cuda()
+    d = sentinel_out((case.M_total, case.N))
+    dg.dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(a, sfa, b, sfb, d, mi)
+    torch.cuda.synchronize()
+    return d
+
+
+def run_masked(dg, case, a=None, sa=None) -> torch.Tensor:
+    a = to_dev_u8(case.a if a is None else a)
+    sfa = dg.sfa_mn_major(to_dev_f32(case.sa if sa is None else sa))
+    b = to_dev_u8(case.b)
+    sfb = to_dev_f32(case.sb)
+    mm = torch.from_numpy(case.masked_m).cuda()
+    d = sentinel_out((case.G, case.M_max, case.N))
+    dg.dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked(a, sfa, b, sfb, d, mm, case.expected_m)
+    torch.cuda.synchronize()
+    return d
+
+
+def sample_rows(M: int, n: int, seed: int) -> np.ndarray:
+    """Rows at tile boundaries (first/last rows of the first, second and last 128-row tiles)
+    plus n seeded random rows."""
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, 127, 128, 129, 255, M - 129, M - 128, M - 2, M - 1]
+    rows = set(r for r in fixed if 0 <= r < M)
+    rows.update(int(r) for r in rng.integers(0, M, size=min(n, M)))
+    return np.array(sorted(rows), dtype=np.int64)
