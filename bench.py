@@ -72,7 +72,12 @@ class Gemm:
         self.shape = dict(kind=kind, M=M, N=N, K=K, G=getattr(c, "G", 1), M_valid=m_valid)
 
 
-def build_workload(name: str):
+def build_workload(name: str, shape=None):
+    if name == "dense":
+        M, N, K = shape
+        c = workloads.dense(M, N, K, seed=6000, a_std=1.0, b_std=0.02)
+        return [Gemm("dense", c, f"dense {M}x{N}x{K}")], \
+            f"dense FP8 NT GEMM M={M} N={N} K={K}, A~N(0,1), B~N(0,0.02)"
     if name == "sweep":
         gemms = []
         for i, (M, N, K) in enumerate(workloads.sweep_shapes()):
@@ -222,7 +227,9 @@ def run_ours(args, rank, world, local_rank):
     import fp8_block_scaled_tma_b200 as dg
 
     torch.cuda.set_device(local_rank)
-    gemms, desc = build_workload(args.workload)
+    gemms, desc = build_workload(args.workload, args.shape)
+    if args.block_n or args.stages:
+        dg.set_config_override(args.block_n, args.stages)
     dev = [DeviceGemm(dg, g) for g in gemms]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
@@ -391,7 +398,7 @@ def run_reference(args):
     """The CPU oracle on a bounded sample of the workload (rank 0 only)."""
     import oracle
     oracle.build()
-    gemms, desc = build_workload(args.workload)
+    gemms, desc = build_workload(args.workload, args.shape)
     cores = os.cpu_count() or 1
     rows = 16
     rng = np.random.default_rng(99)
@@ -420,8 +427,12 @@ def main():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["sweep", "small", "contiguous", "masked", "prefill"],
-                    default="sweep")
+    ap.add_argument("--workload", choices=["sweep", "small", "contiguous", "masked", "prefill",
+                                           "dense"], default="sweep")
+    ap.add_argument("--shape", type=lambda v: tuple(int(x) for x in v.split(",")), default=None,
+                    help="M,N,K of --workload dense")
+    ap.add_argument("--block-n", type=int, default=0, help="tile override (tuning)")
+    ap.add_argument("--stages", type=int, default=0, help="pipeline-stage override (tuning)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -430,6 +441,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.workload == "dense" and (args.shape is None or len(args.shape) != 3):
+        raise SystemExit("--workload dense needs --shape M,N,K")
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -137,16 +137,12 @@ int make_map(CUtensorMap *map, CUtensorMapDataType dt, void *base, uint64_t d0, 
     return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
 }
 
-template <int BN>
-constexpr int stage_bytes()
-{
-    return dg::Cfg<BN>::kStageBytes;
-}
-
 int stage_bytes_rt(int bn)
 {
-    return ((dg::kBlockM * dg::kBlockK + bn * dg::kBlockK + dg::kSfaBytes) + 1023) / 1024 * 1024;
+    return dg::kBlockM * dg::kBlockK + bn * dg::kBlockK;  // A tile + B tile (multiple of 1024)
 }
+
+constexpr int kSfaRingBytes = dg::kSfaSlots * dg::kSfaBytes;
 
 using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, Params);
 
@@ -279,12 +275,13 @@ int launch(const LaunchArgs &args)
             ks.static_bytes = static_cast<int>(fa.sharedSizeBytes);
         }
         const int dyn_cap = info->smem_optin - ks.static_bytes;  // dynamic bytes allowed
-        stages = std::min(dg::kMaxStages, (dyn_cap - 1024) / sbytes);
+        stages = std::min(dg::kMaxStages, (dyn_cap - 1024 - kSfaRingBytes) / sbytes);
         if (stages_override > 0)
             stages = std::min(stages, stages_override);
         if (stages < 2)
             return DG_ERR_UNSUPPORTED;
-        dyn_smem = stages * sbytes + 1024;  // + slack to align the stages to 1024 bytes
+        // operand stages, the A-scale ring, and slack to align the stages to 1024 bytes
+        dyn_smem = stages * sbytes + kSfaRingBytes + 1024;
         dyn_smem = std::min(std::max(dyn_smem, kMinDynSmem), dyn_cap);
         if (ks.limit_set < dyn_smem) {
             cudaError_t e =

@@ -8,8 +8,9 @@
 // "如何使用" (NT dense, MoE contiguous, MoE masked).
 //
 // Blackwell design (one CTA of 384 threads per SM, persistent over output tiles):
-//   warp 0          TMA producer: per K block loads A [128 x 128 B], B [BN x 128 B] (both with
-//                   the 128-byte swizzle) and the 128 fp32 scales of A into one pipeline stage.
+//   warp 0          TMA producer: per K block loads A [128 x 128 B] and B [BN x 128 B] (both with
+//                   the 128-byte swizzle) into one operand stage, and the 128 fp32 scales of A
+//                   into a separate, deeper ring (the operand stage is freed by the MMA alone).
 //   warp 1          allocates tensor memory, then issues 4 x tcgen05.mma kind::f8f6f4 (K = 32
 //                   each) per K block into one of NB TMEM buffers of BN fp32 columns, and
 //                   commits the stage (free) and the buffer (full) to mbarriers.
@@ -36,6 +37,8 @@ constexpr int kNumThreads = 384;
 constexpr int kNumMathWarps = 8;
 constexpr int kFirstMathWarp = 4;
 constexpr int kMaxStages = 8;
+constexpr int kSfaSlots = 16;          // ring of A-scale strips (128 fp32 each), decoupled from the
+                                       // operand stages so that the MMA alone frees a stage
 constexpr int kTmemCols = 512;
 constexpr int kMaxMaskedGroups = 1024;
 constexpr int kSfaBytes = kBlockM * 4;
@@ -70,13 +73,14 @@ template <int BN>
 struct Cfg {
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN must be a multiple of 32 in [32, 256]");
     static constexpr int kCols = BN / 2;                      // columns per promotion thread
-    static constexpr int kChunk = (kCols % 32 == 0) ? 32 : 16;
-    static constexpr int kNumChunks = kCols / kChunk;
+    // The partial of one K block is read from TMEM in one burst when the accumulator and the
+    // partial fit in registers together (kCols <= 96), else in two halves.
+    static constexpr int kPart1 = (kCols <= 96) ? kCols : ((kCols / 2 + 15) / 16 * 16);
     static constexpr int kTmemBufs = (kTmemCols / BN) >= 4 ? 4 : (kTmemCols / BN);
     static constexpr int kABytes = kBlockM * kBlockK;         // 16 KB
     static constexpr int kBBytes = BN * kBlockK;
-    static constexpr int kStageBytes = ((kABytes + kBBytes + kSfaBytes) + 1023) / 1024 * 1024;
-    static constexpr uint32_t kTxBytes = kABytes + kBBytes + kSfaBytes;
+    static constexpr int kStageBytes = kABytes + kBBytes;     // multiple of 1024
+    static constexpr uint32_t kTxBytes = kABytes + kBBytes;
     static constexpr uint32_t kIdesc = ptx::idesc_e4m3_f32(kBlockM, BN);
 };
 
@@ -84,6 +88,8 @@ struct Cfg {
 struct SmemCtl {
     uint64_t full[kMaxStages];
     uint64_t empty[kMaxStages];
+    uint64_t sfa_full[kSfaSlots];
+    uint64_t sfa_empty[kSfaSlots];
     uint64_t tmem_full[4];
     uint64_t tmem_empty[4];
     uint64_t drain;
@@ -210,22 +216,30 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 
     auto stage_a = [&](int s) { return smem_base + s * C::kStageBytes; };
     auto stage_b = [&](int s) { return smem_base + s * C::kStageBytes + C::kABytes; };
-    auto stage_sfa = [&](int s) {
-        return reinterpret_cast<const float *>(smem_gen + s * C::kStageBytes + C::kABytes +
-                                               C::kBBytes);
+    // A-scale ring after the operand stages
+    const int sfa_off = p.stages * C::kStageBytes;
+    auto sfa_slot = [&](int j) { return smem_base + sfa_off + j * kSfaBytes; };
+    auto sfa_ptr = [&](int j) {
+        return reinterpret_cast<const float *>(smem_gen + sfa_off + j * kSfaBytes);
     };
     const uint32_t bar_full = ptx::smem_addr(&ctl.full[0]);
     const uint32_t bar_empty = ptx::smem_addr(&ctl.empty[0]);
     const uint32_t bar_tfull = ptx::smem_addr(&ctl.tmem_full[0]);
     const uint32_t bar_tempty = ptx::smem_addr(&ctl.tmem_empty[0]);
     const uint32_t bar_drain = ptx::smem_addr(&ctl.drain);
+    const uint32_t bar_sfull = ptx::smem_addr(&ctl.sfa_full[0]);
+    const uint32_t bar_sempty = ptx::smem_addr(&ctl.sfa_empty[0]);
     volatile int *abort_flag = &ctl.abort_flag;
 
     // ---- set-up ------------------------------------------------------------------------
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             ptx::mbar_init(bar_full + 8 * s, 1);
-            ptx::mbar_init(bar_empty + 8 * s, 1 + kNumMathWarps);
+            ptx::mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int j = 0; j < kSfaSlots; ++j) {
+            ptx::mbar_init(bar_sfull + 8 * j, 1);
+            ptx::mbar_init(bar_sempty + 8 * j, kNumMathWarps);
         }
         for (int b = 0; b < C::kTmemBufs; ++b) {
             ptx::mbar_init(bar_tfull + 8 * b, 1);
@@ -270,50 +284,81 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 
     if (warp < kFirstMathWarp) {
         ptx::setmaxnreg_dec<40>();
-        if (warp == 0 && lane == 0) {
-            // ---------------- TMA producer ----------------
-            uint32_t it = 0;
-            int s = 0;
-            uint32_t ph = 0;
+        if (warp == 0) {
+            // ---------------- TMA producer (whole warp; one elected lane issues) ----------------
+            uint32_t n_sfa = 0, n_op = 0;  // loads issued into each ring
+            int s = 0, j = 0;
+            uint32_t ph = 0, jph = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
                 Tile ti;
                 if (!resolve_tile<L>(p, ctl, t, ti))
                     continue;
                 const int n0 = ti.n0 * BN;
-                const int a_y = ti.m0;
                 for (int kb = 0; kb < p.num_kb; ++kb) {
-                    if (!wait_one(bar_empty + 8 * s, ph ^ 1, p, abort_flag)) {
+                    // A scales of this K block into the scale ring
+                    if (!__all_sync(0xffffffffu, wait_one(bar_sempty + 8 * j, jph ^ 1, p, abort_flag))) {
                         ok = false;
                         break;
                     }
-                    const uint32_t fb = bar_full + 8 * s;
-                    ptx::mbar_arrive_expect_tx(fb, C::kTxBytes);
-                    ptx::tma_load_3d(stage_a(s), &tmap_a, fb, kb * kBlockK, a_y, ti.a_z);
-                    ptx::tma_load_3d(stage_b(s), &tmap_b, fb, kb * kBlockK, n0, ti.g);
-                    ptx::tma_load_3d(ptx::smem_addr(stage_sfa(s)), &tmap_sfa, fb, ti.m0, kb,
-                                     ti.a_z);
-                    ++it;
+                    if (ptx::elect_one()) {
+                        ptx::mbar_arrive_expect_tx(bar_sfull + 8 * j, kSfaBytes);
+                        ptx::tma_load_3d(sfa_slot(j), &tmap_sfa, bar_sfull + 8 * j, ti.m0, kb, ti.a_z);
+                    }
+                    __syncwarp();
+                    ++n_sfa;
+                    if (++j == kSfaSlots) {
+                        j = 0;
+                        jph ^= 1;
+                    }
+                    // A and B tiles into the operand ring
+                    if (!__all_sync(0xffffffffu, wait_one(bar_empty + 8 * s, ph ^ 1, p, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    if (ptx::elect_one()) {
+                        const uint32_t fb = bar_full + 8 * s;
+                        ptx::mbar_arrive_expect_tx(fb, C::kTxBytes);
+                        ptx::tma_load_3d(stage_a(s), &tmap_a, fb, kb * kBlockK, ti.m0, ti.a_z);
+                        ptx::tma_load_3d(stage_b(s), &tmap_b, fb, kb * kBlockK, n0, ti.g);
+                    }
+                    __syncwarp();
+                    ++n_op;
                     if (++s == p.stages) {
                         s = 0;
                         ph ^= 1;
                     }
                 }
             }
-            // Wind down: every issued load must have landed before the CTA may exit.  The
-            // last min(it, stages) loads are the only ones that can still be in flight.
-            int pending = it < static_cast<uint32_t>(p.stages) ? static_cast<int>(it) : p.stages;
-            int ds = s;
-            uint32_t dph = ph;
-            for (int i = 0; i < pending; ++i) {
-                if (--ds < 0) {
-                    ds = p.stages - 1;
-                    dph ^= 1;
+            // Wind down: every issued load must have landed before the CTA may exit.  In each
+            // ring only the last (ring size) loads can still be in flight; waiting on a slot's
+            // most recent phase returns at once if it was already consumed.
+            {
+                int pending = n_sfa < static_cast<uint32_t>(kSfaSlots) ? static_cast<int>(n_sfa)
+                                                                        : kSfaSlots;
+                int dj = j;
+                uint32_t dph = jph;
+                for (int i = 0; i < pending; ++i) {
+                    if (--dj < 0) {
+                        dj = kSfaSlots - 1;
+                        dph ^= 1;
+                    }
+                    wait_drain(bar_sfull + 8 * dj, dph);
                 }
-                wait_drain(bar_full + 8 * ds, dph);
+                pending = n_op < static_cast<uint32_t>(p.stages) ? static_cast<int>(n_op) : p.stages;
+                int ds = s;
+                dph = ph;
+                for (int i = 0; i < pending; ++i) {
+                    if (--ds < 0) {
+                        ds = p.stages - 1;
+                        dph ^= 1;
+                    }
+                    wait_drain(bar_full + 8 * ds, dph);
+                }
             }
-        } else if (warp == 1 && lane == 0) {
-            // ---------------- MMA issuer ----------------
+            __syncwarp();
+        } else if (warp == 1) {
+            // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
             int s = 0;
             uint32_t ph = 0;
             int buf = 0;
@@ -324,23 +369,27 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 if (!resolve_tile<L>(p, ctl, t, ti))
                     continue;
                 for (int kb = 0; kb < p.num_kb; ++kb) {
-                    if (!wait_one(bar_tempty + 8 * buf, bph ^ 1, p, abort_flag) ||
-                        !wait_one(bar_full + 8 * s, ph, p, abort_flag)) {
+                    bool w = wait_one(bar_tempty + 8 * buf, bph ^ 1, p, abort_flag) &&
+                             wait_one(bar_full + 8 * s, ph, p, abort_flag);
+                    if (!__all_sync(0xffffffffu, w)) {
                         ok = false;
                         break;
                     }
                     ptx::tc_fence_after();
-                    const uint64_t adesc = ptx::sdesc_kmajor_sw128(stage_a(s));
-                    const uint64_t bdesc = ptx::sdesc_kmajor_sw128(stage_b(s));
-                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+                    if (ptx::elect_one()) {
+                        const uint64_t adesc = ptx::sdesc_kmajor_sw128(stage_a(s));
+                        const uint64_t bdesc = ptx::sdesc_kmajor_sw128(stage_b(s));
+                        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
 #pragma unroll
-                    for (int k = 0; k < kBlockK / kUmmaK; ++k) {
-                        // advance the start address by 32 bytes (2 x 16 B) per K step
-                        ptx::mma_f8f6f4(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::kIdesc,
-                                        k > 0 ? 1u : 0u);
+                        for (int k = 0; k < kBlockK / kUmmaK; ++k) {
+                            // advance the start address by 32 bytes (2 x 16 B) per K step
+                            ptx::mma_f8f6f4(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::kIdesc,
+                                            k > 0 ? 1u : 0u);
+                        }
+                        ptx::mma_commit(bar_empty + 8 * s);
+                        ptx::mma_commit(bar_tfull + 8 * buf);
                     }
-                    ptx::mma_commit(bar_empty + 8 * s);
-                    ptx::mma_commit(bar_tfull + 8 * buf);
+                    __syncwarp();
                     if (++s == p.stages) {
                         s = 0;
                         ph ^= 1;
@@ -352,8 +401,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 }
             }
             // Wind down: all issued MMAs complete before tensor memory is released.
-            ptx::mma_commit(bar_drain);
+            if (ptx::elect_one())
+                ptx::mma_commit(bar_drain);
+            __syncwarp();
             wait_drain(bar_drain, 0);
+            __syncwarp();
         }
     } else {
         ptx::setmaxnreg_inc<232>();
@@ -364,8 +416,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const int row = q * 32 + lane;            // row within the tile
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    static_cast<uint32_t>(half * C::kCols);
-        int s = 0;
-        uint32_t ph = 0;
+        constexpr int P1 = C::kPart1;             // columns loaded before the first wait
+        constexpr int P2 = C::kCols - P1;         // columns loaded after it (0 if all at once)
+        int j = 0;
+        uint32_t jph = 0;
         int buf = 0;
         uint32_t bph = 0;
         bool ok = true;
@@ -375,108 +429,81 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 continue;
             const int n0 = ti.n0 * BN;
             const int col0 = n0 + half * C::kCols;  // first global column of this thread
-            // the (at most two) 128-column scale blocks of B this thread's columns touch
+            // the (at most two) 128-column scale blocks of B this thread's columns touch; the
+            // boundary (if any) lies on a 16-column group edge
             const int nb_lo = min(col0 / kBlockK, p.num_nb - 1);
             const int nb_hi = min((col0 + C::kCols - 1) / kBlockK, p.num_nb - 1);
-            uint32_t hi_mask = 0;
-#pragma unroll
-            for (int j = 0; j < C::kCols / 16; ++j)
-                if ((col0 + 16 * j) / kBlockK > nb_lo)
-                    hi_mask |= 1u << j;
+            const int split = min(C::kCols, max(0, (nb_lo + 1) * kBlockK - col0));  // first hi column
             const float *sfb_lo = p.sfb + (static_cast<size_t>(ti.g) * p.num_nb + nb_lo) * p.num_kb;
             const float *sfb_hi = p.sfb + (static_cast<size_t>(ti.g) * p.num_nb + nb_hi) * p.num_kb;
 
             float acc[C::kCols];
 #pragma unroll
-            for (int j = 0; j < C::kCols; ++j)
-                acc[j] = 0.0f;
+            for (int c = 0; c < C::kCols; ++c)
+                acc[c] = 0.0f;
 
+            float sb_lo = __ldg(sfb_lo);
+            float sb_hi = __ldg(sfb_hi);
             for (int kb = 0; kb < p.num_kb; ++kb) {
-                const float sb_lo = __ldg(sfb_lo + kb);
-                const float sb_hi = __ldg(sfb_hi + kb);
-                bool w = wait_one(bar_full + 8 * s, ph, p, abort_flag) &&
+                // prefetch the B scales of the next K block
+                const int kn = kb + 1 < p.num_kb ? kb + 1 : kb;
+                const float sb_lo_next = __ldg(sfb_lo + kn);
+                const float sb_hi_next = __ldg(sfb_hi + kn);
+                bool w = wait_one(bar_sfull + 8 * j, jph, p, abort_flag) &&
                          wait_one(bar_tfull + 8 * buf, bph, p, abort_flag);
-                w = __all_sync(0xffffffffu, w);
-                if (!w) {
+                if (!__all_sync(0xffffffffu, w)) {
                     ok = false;
                     break;
                 }
                 ptx::tc_fence_after();
-                const float sa = stage_sfa(s)[row];
+                const uint32_t taddr = lane_base + static_cast<uint32_t>(buf * BN);
+                uint32_t pr[P1];
+                ptx::tmem_ld_cols<P1>(taddr, pr);
+                const float sa = sfa_ptr(j)[row];
                 const float scale_lo = sa * sb_lo;
                 const float scale_hi = sa * sb_hi;
-                const uint32_t taddr = lane_base + static_cast<uint32_t>(buf * BN);
-
-                uint32_t r0[16], r1[16];
-                if (C::kChunk == 32) {
-                    uint32_t r2[16], r3[16];
-                    ptx::tmem_ld_x16(taddr, r0);
-                    ptx::tmem_ld_x16(taddr + 16, r1);
-                    ptx::tmem_wait_ld(r0);
-                    ptx::tmem_wait_ld(r1);
-#pragma unroll
-                    for (int c = 0; c < C::kNumChunks; ++c) {
-                        if (c + 1 < C::kNumChunks) {
-                            ptx::tmem_ld_x16(taddr + 32 * (c + 1), r2);
-                            ptx::tmem_ld_x16(taddr + 32 * (c + 1) + 16, r3);
-                        } else {
-                            // all partials of this K block are in registers: free the buffer
-                            ptx::tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) {
-                                ptx::mbar_arrive(bar_tempty + 8 * buf);
-                                ptx::mbar_arrive(bar_empty + 8 * s);
-                            }
-                        }
-                        const float sc0 = ((hi_mask >> (2 * c)) & 1u) ? scale_hi : scale_lo;
-                        const float sc1 = ((hi_mask >> (2 * c + 1)) & 1u) ? scale_hi : scale_lo;
-#pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            acc[32 * c + j] = fmaf(__uint_as_float(r0[j]), sc0, acc[32 * c + j]);
-#pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            acc[32 * c + 16 + j] =
-                                fmaf(__uint_as_float(r1[j]), sc1, acc[32 * c + 16 + j]);
-                        if (c + 1 < C::kNumChunks) {
-                            ptx::tmem_wait_ld(r2);
-                            ptx::tmem_wait_ld(r3);
-#pragma unroll
-                            for (int j = 0; j < 16; ++j) {
-                                r0[j] = r2[j];
-                                r1[j] = r3[j];
-                            }
-                        }
-                    }
-                } else {
-                    ptx::tmem_ld_x16(taddr, r0);
-                    ptx::tmem_wait_ld(r0);
-#pragma unroll
-                    for (int c = 0; c < C::kNumChunks; ++c) {
-                        if (c + 1 < C::kNumChunks) {
-                            ptx::tmem_ld_x16(taddr + 16 * (c + 1), r1);
-                        } else {
-                            ptx::tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) {
-                                ptx::mbar_arrive(bar_tempty + 8 * buf);
-                                ptx::mbar_arrive(bar_empty + 8 * s);
-                            }
-                        }
-                        const float sc = ((hi_mask >> c) & 1u) ? scale_hi : scale_lo;
-#pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            acc[16 * c + j] = fmaf(__uint_as_float(r0[j]), sc, acc[16 * c + j]);
-                        if (c + 1 < C::kNumChunks) {
-                            ptx::tmem_wait_ld(r1);
-#pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                r0[j] = r1[j];
-                        }
+                ptx::tmem_wait_cols<P1>(pr);
+                if (P2 == 0) {
+                    // the whole partial is in registers: free the TMEM buffer and scale slot
+                    // before doing the arithmetic
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        ptx::mbar_arrive(bar_tempty + 8 * buf);
+                        ptx::mbar_arrive(bar_sempty + 8 * j);
                     }
                 }
-                if (++s == p.stages) {
-                    s = 0;
-                    ph ^= 1;
+#pragma unroll
+                for (int g16 = 0; g16 < P1 / 16; ++g16) {
+                    const float sc = (16 * g16 >= split) ? scale_hi : scale_lo;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        acc[16 * g16 + e] = fmaf(__uint_as_float(pr[16 * g16 + e]), sc, acc[16 * g16 + e]);
+                }
+                if (P2 > 0) {
+                    // second part reuses the same registers
+                    ptx::tmem_ld_cols<(P2 > 0 ? P2 : 16)>(taddr + P1, pr);
+                    ptx::tmem_wait_cols<(P2 > 0 ? P2 : 16)>(pr);
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        ptx::mbar_arrive(bar_tempty + 8 * buf);
+                        ptx::mbar_arrive(bar_sempty + 8 * j);
+                    }
+#pragma unroll
+                    for (int g16 = 0; g16 < P2 / 16; ++g16) {
+                        const float sc = (P1 + 16 * g16 >= split) ? scale_hi : scale_lo;
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            acc[P1 + 16 * g16 + e] =
+                                fmaf(__uint_as_float(pr[16 * g16 + e]), sc, acc[P1 + 16 * g16 + e]);
+                    }
+                }
+                sb_lo = sb_lo_next;
+                sb_hi = sb_hi_next;
+                if (++j == kSfaSlots) {
+                    j = 0;
+                    jph ^= 1;
                 }
                 if (++buf == C::kTmemBufs) {
                     buf = 0;
