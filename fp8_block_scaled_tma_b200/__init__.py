@@ -69,6 +69,8 @@ def _load() -> ctypes.CDLL:
     lib.dg_set_wait_timeout_ns.restype = ctypes.c_ulonglong
     lib.dg_set_config_override.argtypes = [i, i]
     lib.dg_set_config_override.restype = i
+    lib.dg_set_pair_mode.argtypes = [i]
+    lib.dg_set_pair_mode.restype = i
     ipp = ctypes.POINTER(ctypes.c_int)
     lib.dg_get_last_launch.argtypes = [ipp, ipp, ipp, ipp]
     lib.dg_get_last_launch.restype = i
@@ -161,6 +163,14 @@ def set_wait_timeout_ns(ns: int) -> int:
 
 def set_config_override(block_n: int = 0, num_stages: int = 0) -> None:
     _check(lib.dg_set_config_override(int(block_n), int(num_stages)), "dg_set_config_override")
+
+
+def set_pair_mode(mode: int) -> int:
+    """0 automatic, 1 one-CTA kernels only, 2 CTA-pair kernels where the layout allows."""
+    r = lib.dg_set_pair_mode(int(mode))
+    if r < 0:
+        raise DGError(r, "dg_set_pair_mode")
+    return r
 
 
 def get_last_launch() -> dict:

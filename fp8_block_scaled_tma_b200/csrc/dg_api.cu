@@ -12,6 +12,7 @@
 
 #include "../../include/dg.h"
 #include "dg_kernel.cuh"
+#include "dg_pair_kernel.cuh"
 
 namespace {
 
@@ -37,7 +38,9 @@ struct KernelSmem {
     int static_bytes = -1;  // static shared memory of the kernel
     int limit_set = 0;      // dynamic shared-memory limit already set on this device
 };
-KernelSmem g_smem[kMaxDevices][3][8];  // per device / layout / BN
+KernelSmem g_smem[kMaxDevices][3][8];       // 1-CTA kernels, per device / layout / BN
+KernelSmem g_smem_pair[kMaxDevices][3][8];  // CTA-pair kernels
+int g_pair_mode = 0;                        // 0 auto, 1 single-CTA kernels only, 2 pairs where possible
 int g_num_sms_cap = 0;
 unsigned long long g_timeout_ns = kDefaultTimeoutNs;
 int g_override_bn = 0;
@@ -46,7 +49,7 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 struct LastLaunch {
     bool valid = false;
-    int block_n = 0, stages = 0, grid = 0, tiles = 0;
+    int block_n = 0, stages = 0, grid = 0, tiles = 0, pair = 0;
 };
 thread_local LastLaunch t_last;
 
@@ -142,9 +145,77 @@ int stage_bytes_rt(int bn)
     return dg::kBlockM * dg::kBlockK + bn * dg::kBlockK;  // A tile + B tile (multiple of 1024)
 }
 
-constexpr int kSfaRingBytes = dg::kSfaSlots * dg::kSfaBytes;
 
-using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, Params);
+using KernelFn = void (*)(CUtensorMap, CUtensorMap, Params);
+
+// 4-D view [groups][K/128][rows][128 bytes] of a K-major uint8 operand: one box holds `kbs`
+// consecutive 128-wide K blocks of `box_rows` rows, laid out K block by K block in shared memory.
+int make_map_kblocks(CUtensorMap *map, void *base, uint64_t K, uint64_t rows, uint64_t groups,
+                     uint32_t box_rows, uint32_t kbs)
+{
+    cuuint64_t dims[4] = {128, rows, K / 128, groups};
+    cuuint64_t strides[3] = {K, 128, K * rows};
+    cuuint32_t box[4] = {128, box_rows, kbs, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, base, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
+}
+
+template <int L, int BN>
+void *pair_kernel_ptr()
+{
+    return reinterpret_cast<void *>(&dg::dg_gemm_pair_kernel<L, BN>);
+}
+
+void *pick_pair_kernel(int layout, int bn)
+{
+#define DG_PCASE(BNV)                                                                          \
+    case BNV:                                                                                  \
+        return layout == dg::kDense ? pair_kernel_ptr<dg::kDense, BNV>()                        \
+                                    : pair_kernel_ptr<dg::kMasked, BNV>();
+    if (layout == dg::kContiguous)
+        return nullptr;
+    switch (bn) {
+        DG_PCASE(128)
+        DG_PCASE(160)
+        DG_PCASE(192)
+        DG_PCASE(224)
+        DG_PCASE(256)
+    default:
+        return nullptr;
+    }
+#undef DG_PCASE
+}
+
+int pair_stage_bytes(int bn)
+{
+    return dg::kKbPerStage * (dg::kBlockM * dg::kBlockK + bn / 2 * dg::kBlockK);
+}
+
+constexpr int kPairSfaRingBytes = dg::kSfaSlots * dg::kKbPerStage * dg::kBlockM * 4;
+
+// Tile heuristic of the pair kernel: 256-row pair tiles, waves over SM pairs.
+int choose_pair_block_n(long long pair_row_tiles, int N, int num_pairs)
+{
+    int best_bn = 256;
+    double best = 1e300;
+    for (int bn = 128; bn <= 256; bn += 32) {
+        long long n_tiles = (N + bn - 1) / bn;
+        long long tiles = n_tiles * pair_row_tiles;
+        long long waves = (tiles + num_pairs - 1) / num_pairs;
+        double per_tile = static_cast<double>(bn) + 16.0;
+        double t = waves * per_tile;
+        double waste = static_cast<double>(n_tiles * bn - N) / N;
+        t *= 1.0 + 0.5 * waste;
+        if (t < best - 1e-9 || (std::abs(t - best) <= 1e-9 && bn > best_bn)) {
+            best = t;
+            best_bn = bn;
+        }
+    }
+    return best_bn;
+}
 
 template <int L, int BN>
 void *kernel_ptr()
@@ -214,6 +285,141 @@ struct LaunchArgs {
     void *stream;
 };
 
+int launch_pair(const LaunchArgs &args, int dev, DeviceInfo *info, int sms, int bn,
+                int stages_override, unsigned long long timeout)
+{
+    const int M = args.M, N = args.N, K = args.K, G = args.G;
+    const int num_kb = K / dg::kBlockK;
+    const int num_nb = (N + dg::kBlockK - 1) / dg::kBlockK;
+    const int pair_m_tiles = (M + 2 * dg::kBlockM - 1) / (2 * dg::kBlockM);
+    const int num_pairs = sms / 2;
+    if (bn == 0) {
+        long long row_tiles = pair_m_tiles;
+        if (args.layout == dg::kMasked) {
+            int em = args.expected_m > 0 ? std::min(args.expected_m, M) : M;
+            row_tiles = static_cast<long long>(G) * ((em + 2 * dg::kBlockM - 1) / (2 * dg::kBlockM));
+        }
+        bn = choose_pair_block_n(std::max<long long>(1, row_tiles), N, num_pairs);
+    }
+    void *fn = pick_pair_kernel(args.layout, bn);
+    if (fn == nullptr)
+        return DG_ERR_INVALID_ARG;
+    const int n_tiles = (N + bn - 1) / bn;
+    const int sbytes = pair_stage_bytes(bn);
+    int stages = 0, dyn_smem = 0;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        KernelSmem &ks = g_smem_pair[dev][args.layout][bn / 32 - 1];
+        if (ks.static_bytes < 0) {
+            cudaFuncAttributes fa;
+            cudaError_t e = cudaFuncGetAttributes(&fa, fn);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                return DG_ERR_CUDA;
+            }
+            ks.static_bytes = static_cast<int>(fa.sharedSizeBytes);
+        }
+        const int dyn_cap = info->smem_optin - ks.static_bytes;
+        stages = std::min(dg::kMaxStages, (dyn_cap - 1024 - kPairSfaRingBytes) / sbytes);
+        if (stages_override > 0)
+            stages = std::min(stages, stages_override);
+        if (stages < 2)
+            return DG_ERR_UNSUPPORTED;
+        // operand stages, the A-scale ring, and slack to align the stages to 1024 bytes
+        dyn_smem = stages * sbytes + kPairSfaRingBytes + 1024;
+        dyn_smem = std::min(std::max(dyn_smem, kMinDynSmem), dyn_cap);
+        if (ks.limit_set < dyn_smem) {
+            cudaError_t e =
+                cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                return DG_ERR_CUDA;
+            }
+            ks.limit_set = dyn_smem;
+        }
+    }
+
+    const int a_groups = (args.layout == dg::kMasked) ? G : 1;
+    const int b_groups = (args.layout == dg::kDense) ? 1 : G;
+    const int m4 = align4(M);
+    CUtensorMap map_a, map_b, map_sfa;
+    if (make_map_kblocks(&map_a, const_cast<void *>(args.a), K, M, a_groups, dg::kBlockM,
+                         dg::kKbPerStage) != DG_OK ||
+        make_map_kblocks(&map_b, const_cast<void *>(args.b), K, N, b_groups, bn / 2,
+                         dg::kKbPerStage) != DG_OK ||
+        // A scales [groups][K/128][align4(rows)]: one box = 128 rows x kKbPerStage K blocks
+        make_map(&map_sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float *>(args.sfa), m4,
+                 num_kb, a_groups, static_cast<uint64_t>(m4) * 4,
+                 static_cast<uint64_t>(m4) * 4 * num_kb, dg::kBlockM, dg::kKbPerStage,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) != DG_OK) {
+        if (debug_enabled())
+            std::fprintf(stderr, "[dg] cuTensorMapEncodeTiled failed (pair)\n");
+        return DG_ERR_CUDA;
+    }
+
+    Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.G = (args.layout == dg::kDense) ? 1 : G;
+    p.num_kb = num_kb;
+    p.num_nb = num_nb;
+    p.m_tiles = pair_m_tiles;
+    p.n_tiles = n_tiles;
+    p.stages = stages;
+    p.raster_m = 8;
+    p.sfa = args.sfa;
+    p.sfa_ld = m4;
+    p.sfb = args.sfb;
+    p.d = static_cast<__nv_bfloat16 *>(args.d);
+    p.m_indices = nullptr;
+    p.masked_m = args.masked_m;
+    p.err = info->err_ptr;
+    p.timeout_ns = timeout;
+    long long tiles = (args.layout == dg::kMasked)
+                          ? static_cast<long long>(G) * pair_m_tiles * n_tiles
+                          : static_cast<long long>(pair_m_tiles) * n_tiles;
+    if (tiles > 0x7FFFFFFFLL)
+        return DG_ERR_INVALID_ARG;
+    p.num_tiles = static_cast<int>(tiles);
+    const int pairs = static_cast<int>(std::min<long long>(num_pairs, tiles));
+    if (pairs <= 0)
+        return DG_OK;
+
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(dg::kNumThreads, 1, 1);
+    cfg.dynamicSmemBytes = dyn_smem;
+    cfg.stream = static_cast<cudaStream_t>(args.stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void *kargs[] = {&map_a, &map_b, &map_sfa, &p};
+    cudaError_t e = cudaLaunchKernelExC(&cfg, fn, kargs);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        if (debug_enabled())
+            std::fprintf(stderr, "[dg] pair launch failed: %s\n", cudaGetErrorString(e));
+        return DG_ERR_CUDA;
+    }
+    t_last.valid = true;
+    t_last.block_n = bn;
+    t_last.stages = stages;
+    t_last.grid = 2 * pairs;
+    t_last.tiles = p.num_tiles;
+    t_last.pair = 1;
+    if (debug_enabled())
+        std::fprintf(stderr, "[dg] pair layout=%d M=%d N=%d K=%d G=%d BN=%d stages=%d grid=%d tiles=%d smem=%d\n",
+                     args.layout, M, N, K, G, bn, stages, 2 * pairs, p.num_tiles, dyn_smem);
+    return DG_OK;
+}
+
 int launch(const LaunchArgs &args)
 {
     int dev = 0;
@@ -237,12 +443,29 @@ int launch(const LaunchArgs &args)
     int bn;
     int stages_override;
     unsigned long long timeout;
+    int pair_mode;
     {
         std::lock_guard<std::mutex> lock(g_mutex);
         bn = g_override_bn;
         stages_override = g_override_stages;
         timeout = g_timeout_ns;
+        pair_mode = g_pair_mode;
     }
+    // CTA pairs (cta_group::2) for the dense and masked layouts: 256-row tiles whose B half is
+    // loaded by each CTA.  Auto mode uses them when a tile of 256 rows is mostly useful.
+    bool use_pair = false;
+    if (args.layout != dg::kContiguous && sms >= 2 && pair_mode != 1) {
+        if (pair_mode == 2)
+            use_pair = true;
+        else if (args.layout == dg::kDense)
+            use_pair = M > 192;
+        else
+            use_pair = args.expected_m == 0 || args.expected_m > 64;
+        if (bn != 0 && pick_pair_kernel(args.layout, bn) == nullptr)
+            use_pair = false;  // the block_n override names a tile the pair kernel lacks
+    }
+    if (use_pair)
+        return launch_pair(args, dev, info, sms, bn, stages_override, timeout);
     if (bn == 0) {
         long long row_tiles = m_tiles;
         if (args.layout == dg::kMasked) {
@@ -275,13 +498,12 @@ int launch(const LaunchArgs &args)
             ks.static_bytes = static_cast<int>(fa.sharedSizeBytes);
         }
         const int dyn_cap = info->smem_optin - ks.static_bytes;  // dynamic bytes allowed
-        stages = std::min(dg::kMaxStages, (dyn_cap - 1024 - kSfaRingBytes) / sbytes);
+        stages = std::min(dg::kMaxStages, (dyn_cap - 1024) / sbytes);
         if (stages_override > 0)
             stages = std::min(stages, stages_override);
         if (stages < 2)
             return DG_ERR_UNSUPPORTED;
-        // operand stages, the A-scale ring, and slack to align the stages to 1024 bytes
-        dyn_smem = stages * sbytes + kSfaRingBytes + 1024;
+        dyn_smem = stages * sbytes + 1024;  // + slack to align the stages to 1024 bytes
         dyn_smem = std::min(std::max(dyn_smem, kMinDynSmem), dyn_cap);
         if (ks.limit_set < dyn_smem) {
             cudaError_t e =
@@ -302,17 +524,13 @@ int launch(const LaunchArgs &args)
     const int a_groups = (args.layout == dg::kMasked) ? G : 1;
     const int b_groups = (args.layout == dg::kDense) ? 1 : G;
     const int m4 = align4(M);
-    CUtensorMap map_a, map_b, map_sfa;
+    CUtensorMap map_a, map_b;
     if (make_map(&map_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<void *>(args.a), K, a_rows,
                  a_groups, static_cast<uint64_t>(K), static_cast<uint64_t>(K) * a_rows, dg::kBlockK,
                  dg::kBlockM, CU_TENSOR_MAP_SWIZZLE_128B) != DG_OK ||
         make_map(&map_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<void *>(args.b), K, N, b_groups,
                  static_cast<uint64_t>(K), static_cast<uint64_t>(K) * N, dg::kBlockK, bn,
-                 CU_TENSOR_MAP_SWIZZLE_128B) != DG_OK ||
-        make_map(&map_sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float *>(args.sfa), m4,
-                 num_kb, a_groups, static_cast<uint64_t>(m4) * 4,
-                 static_cast<uint64_t>(m4) * 4 * num_kb, dg::kBlockM, 1,
-                 CU_TENSOR_MAP_SWIZZLE_NONE) != DG_OK) {
+                 CU_TENSOR_MAP_SWIZZLE_128B) != DG_OK) {
         if (debug_enabled())
             std::fprintf(stderr, "[dg] cuTensorMapEncodeTiled failed\n");
         return DG_ERR_CUDA;
@@ -330,6 +548,8 @@ int launch(const LaunchArgs &args)
     p.n_tiles = n_tiles;
     p.stages = stages;
     p.raster_m = 16;
+    p.sfa = args.sfa;
+    p.sfa_ld = m4;
     p.sfb = args.sfb;
     p.d = static_cast<__nv_bfloat16 *>(args.d);
     p.m_indices = args.m_indices;
@@ -356,7 +576,7 @@ int launch(const LaunchArgs &args)
     cfg.stream = static_cast<cudaStream_t>(args.stream);
     cfg.attrs = nullptr;
     cfg.numAttrs = 0;
-    void *kargs[] = {&map_a, &map_b, &map_sfa, &p};
+    void *kargs[] = {&map_a, &map_b, &p};
     cudaError_t e = cudaLaunchKernelExC(&cfg, fn, kargs);
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -369,6 +589,7 @@ int launch(const LaunchArgs &args)
     t_last.stages = stages;
     t_last.grid = grid;
     t_last.tiles = p.num_tiles;
+    t_last.pair = 0;
     if (debug_enabled())
         std::fprintf(stderr, "[dg] layout=%d M=%d N=%d K=%d G=%d BN=%d stages=%d grid=%d tiles=%d smem=%d\n",
                      args.layout, M, N, K, G, bn, stages, grid, p.num_tiles, dyn_smem);
@@ -558,6 +779,16 @@ int dg_set_config_override(int block_n, int num_stages)
     g_override_bn = block_n;
     g_override_stages = num_stages;
     return DG_OK;
+}
+
+int dg_set_pair_mode(int mode)
+{
+    if (mode < 0 || mode > 2)
+        return DG_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int prev = g_pair_mode;
+    g_pair_mode = mode;
+    return prev;
 }
 
 int dg_get_last_launch(int *block_n, int *num_stages, int *grid, int *num_tiles)

@@ -9,14 +9,16 @@
 //
 // Blackwell design (one CTA of 384 threads per SM, persistent over output tiles):
 //   warp 0          TMA producer: per K block loads A [128 x 128 B] and B [BN x 128 B] (both with
-//                   the 128-byte swizzle) into one operand stage, and the 128 fp32 scales of A
-//                   into a separate, deeper ring (the operand stage is freed by the MMA alone).
+//                   the 128-byte swizzle) into one operand stage.  Each TMA copy costs the copy
+//                   engine a fixed amount of time besides its bytes, so the small fp32 scales
+//                   are not copied by TMA: the promotion threads read them from global memory.
 //   warp 1          allocates tensor memory, then issues 4 x tcgen05.mma kind::f8f6f4 (K = 32
 //                   each) per K block into one of NB TMEM buffers of BN fp32 columns, and
 //                   commits the stage (free) and the buffer (full) to mbarriers.
 //   warps 4..11     promotion: each thread owns one output row (its TMEM lane) and BN/2
 //                   columns; per K block it loads the fresh partial from TMEM, frees the
-//                   buffer, and adds partial * sa[row] * sb[block] into fp32 registers.  After
+//                   buffer, and adds partial * sa[row] * sb[block] into fp32 registers (sa and
+//                   sb are read with plain loads two K blocks ahead).  After
 //                   the last K block it rounds to bf16 and stores its row segment.
 // Every wait is bounded by a %globaltimer limit; on expiry the kernel records DG_ERR_TIMEOUT,
 // drains its outstanding copies and MMAs, frees tensor memory and returns.
@@ -37,11 +39,8 @@ constexpr int kNumThreads = 384;
 constexpr int kNumMathWarps = 8;
 constexpr int kFirstMathWarp = 4;
 constexpr int kMaxStages = 8;
-constexpr int kSfaSlots = 16;          // ring of A-scale strips (128 fp32 each), decoupled from the
-                                       // operand stages so that the MMA alone frees a stage
 constexpr int kTmemCols = 512;
 constexpr int kMaxMaskedGroups = 1024;
-constexpr int kSfaBytes = kBlockM * 4;
 constexpr uint64_t kDrainTimeoutNs = 1000000000ull;  // fixed bound for the wind-down waits
 
 constexpr int kErrTimeout = -4;
@@ -61,6 +60,8 @@ struct Params {
     int num_tiles;  // dense / contiguous: m_tiles * n_tiles; masked: computed on the device
     int stages;
     int raster_m;   // m-tiles per raster band (dense / contiguous)
+    const float *sfa;   // A scales, MN-major: sfa[(a_z * num_kb + kb) * sfa_ld + row]
+    int sfa_ld;         // align4(rows of a group)
     const float *sfb;
     __nv_bfloat16 *d;
     const int *m_indices;
@@ -85,6 +86,8 @@ struct Cfg {
 };
 
 // Static shared memory: barriers and the bookkeeping words.
+constexpr int kSfaSlots = 8;  // A-scale ring of the CTA-pair kernel (one slot per stage)
+
 struct SmemCtl {
     uint64_t full[kMaxStages];
     uint64_t empty[kMaxStages];
@@ -198,11 +201,121 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity)
     return true;
 }
 
+// Scales a promotion thread needs for one K block: sa of its row and sb of the (at most two)
+// 128-column blocks of B its columns touch.
+struct KbScales {
+    float sa, lo, hi;
+};
+
+__device__ __forceinline__ void load_kb_scales(KbScales &s, const float *sa_ptr, const float *sb_lo,
+                                               const float *sb_hi, int ld, int kb, int nkb)
+{
+    kb = kb < nkb ? kb : nkb - 1;
+    s.sa = __ldg(sa_ptr + static_cast<size_t>(kb) * ld);
+    s.lo = __ldg(sb_lo + kb);
+    s.hi = __ldg(sb_hi + kb);
+}
+
+// Promotion of one K block by one thread: waits for the partial in TMEM buffer `buf`, reads the
+// thread's kCols columns (in one burst when P2 == 0, else in two), frees the buffer by arriving
+// on `release_bar` (a cluster address when `remote`), and adds partial * sa * sb into acc.
+// Columns >= split use the higher B scale block.  Returns false when the wait gave up.
+// The scale products are formed after the TMEM wait so that a late scale never delays the
+// release of the buffer.
+template <int P1, int P2, int NCOLS>
+__device__ __forceinline__ bool promote_kb(float (&acc)[NCOLS], float sa, float sb_lo, float sb_hi,
+                                           uint32_t taddr, uint32_t full_bar, uint32_t parity,
+                                           uint32_t release_bar, bool remote, int split,
+                                           int lane, const Params &p, volatile int *abort_flag)
+{
+    if (!__all_sync(0xffffffffu, wait_one(full_bar, parity, p, abort_flag)))
+        return false;
+    ptx::tc_fence_after();
+    uint32_t pr[P1];
+    ptx::tmem_ld_cols<P1>(taddr, pr);
+    ptx::tmem_wait_cols<P1>(pr);
+    auto release = [&]() {
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+            if (remote)
+                ptx::mbar_arrive_cluster(release_bar);
+            else
+                ptx::mbar_arrive(release_bar);
+        }
+    };
+    if (P2 == 0)
+        release();  // the whole partial is in registers: free the buffer before the arithmetic
+    const float scale_lo = sa * sb_lo;
+    const float scale_hi = sa * sb_hi;
+#pragma unroll
+    for (int g16 = 0; g16 < P1 / 16; ++g16) {
+        const float f = (16 * g16 >= split) ? scale_hi : scale_lo;
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            acc[16 * g16 + e] = fmaf(__uint_as_float(pr[16 * g16 + e]), f, acc[16 * g16 + e]);
+    }
+    if (P2 > 0) {
+        // second part reuses the same registers
+        ptx::tmem_ld_cols<(P2 > 0 ? P2 : 16)>(taddr + P1, pr);
+        ptx::tmem_wait_cols<(P2 > 0 ? P2 : 16)>(pr);
+        release();
+#pragma unroll
+        for (int g16 = 0; g16 < P2 / 16; ++g16) {
+            const float f = (P1 + 16 * g16 >= split) ? scale_hi : scale_lo;
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                acc[P1 + 16 * g16 + e] = fmaf(__uint_as_float(pr[16 * g16 + e]), f, acc[P1 + 16 * g16 + e]);
+        }
+    }
+    return true;
+}
+
+// The K loop of a promotion thread for one tile.  It is unrolled by two with two named scale
+// sets, each reloaded right after its use, so a scale load has a whole K block to land and no
+// register move waits on it.  `tbuf_release(buf)` gives the barrier address that frees buffer
+// `buf` (and whether it is remote).
+template <int BN, int P1, int P2, int NCOLS, int NBUF, class Release>
+__device__ __forceinline__ bool promote_tile(float (&acc)[NCOLS], const float *sa_ptr,
+                                             const float *sb_lo, const float *sb_hi,
+                                             uint32_t lane_base, uint32_t bar_tfull, int &buf,
+                                             uint32_t &bph, Release tbuf_release, int split,
+                                             int lane, const Params &p, volatile int *abort_flag)
+{
+    KbScales s0, s1;
+    load_kb_scales(s0, sa_ptr, sb_lo, sb_hi, p.sfa_ld, 0, p.num_kb);
+    load_kb_scales(s1, sa_ptr, sb_lo, sb_hi, p.sfa_ld, 1, p.num_kb);
+    auto step = [&](const KbScales &sc) -> bool {
+        uint32_t rel;
+        bool remote;
+        tbuf_release(buf, rel, remote);
+        const bool ok = promote_kb<P1, P2>(acc, sc.sa, sc.lo, sc.hi,
+                                           lane_base + static_cast<uint32_t>(buf * BN),
+                                           bar_tfull + 8 * buf, bph, rel, remote, split, lane, p,
+                                           abort_flag);
+        if (++buf == NBUF) {
+            buf = 0;
+            bph ^= 1;
+        }
+        return ok;
+    };
+    for (int kb = 0; kb < p.num_kb; kb += 2) {
+        if (!step(s0))
+            return false;
+        load_kb_scales(s0, sa_ptr, sb_lo, sb_hi, p.sfa_ld, kb + 2, p.num_kb);
+        if (kb + 1 < p.num_kb) {
+            if (!step(s1))
+                return false;
+            load_kb_scales(s1, sa_ptr, sb_lo, sb_hi, p.sfa_ld, kb + 3, p.num_kb);
+        }
+    }
+    return true;
+}
+
 template <int L, int BN>
 __global__ void __launch_bounds__(kNumThreads, 1)
     dg_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                   const __grid_constant__ CUtensorMap tmap_b,
-                   const __grid_constant__ CUtensorMap tmap_sfa, const Params p)
+                   const __grid_constant__ CUtensorMap tmap_b, const Params p)
 {
     using C = Cfg<BN>;
     __shared__ SmemCtl ctl;
@@ -216,19 +329,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 
     auto stage_a = [&](int s) { return smem_base + s * C::kStageBytes; };
     auto stage_b = [&](int s) { return smem_base + s * C::kStageBytes + C::kABytes; };
-    // A-scale ring after the operand stages
-    const int sfa_off = p.stages * C::kStageBytes;
-    auto sfa_slot = [&](int j) { return smem_base + sfa_off + j * kSfaBytes; };
-    auto sfa_ptr = [&](int j) {
-        return reinterpret_cast<const float *>(smem_gen + sfa_off + j * kSfaBytes);
-    };
     const uint32_t bar_full = ptx::smem_addr(&ctl.full[0]);
     const uint32_t bar_empty = ptx::smem_addr(&ctl.empty[0]);
     const uint32_t bar_tfull = ptx::smem_addr(&ctl.tmem_full[0]);
     const uint32_t bar_tempty = ptx::smem_addr(&ctl.tmem_empty[0]);
     const uint32_t bar_drain = ptx::smem_addr(&ctl.drain);
-    const uint32_t bar_sfull = ptx::smem_addr(&ctl.sfa_full[0]);
-    const uint32_t bar_sempty = ptx::smem_addr(&ctl.sfa_empty[0]);
     volatile int *abort_flag = &ctl.abort_flag;
 
     // ---- set-up ------------------------------------------------------------------------
@@ -236,10 +341,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         for (int s = 0; s < p.stages; ++s) {
             ptx::mbar_init(bar_full + 8 * s, 1);
             ptx::mbar_init(bar_empty + 8 * s, 1);
-        }
-        for (int j = 0; j < kSfaSlots; ++j) {
-            ptx::mbar_init(bar_sfull + 8 * j, 1);
-            ptx::mbar_init(bar_sempty + 8 * j, kNumMathWarps);
         }
         for (int b = 0; b < C::kTmemBufs; ++b) {
             ptx::mbar_init(bar_tfull + 8 * b, 1);
@@ -250,7 +351,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tmap_a);
         ptx::prefetch_tmap(&tmap_b);
-        ptx::prefetch_tmap(&tmap_sfa);
     }
     if (warp == 1) {
         ptx::tmem_alloc(ptx::smem_addr(&ctl.tmem_base), kTmemCols);
@@ -286,9 +386,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         ptx::setmaxnreg_dec<40>();
         if (warp == 0) {
             // ---------------- TMA producer (whole warp; one elected lane issues) ----------------
-            uint32_t n_sfa = 0, n_op = 0;  // loads issued into each ring
-            int s = 0, j = 0;
-            uint32_t ph = 0, jph = 0;
+            uint32_t n_op = 0;  // operand loads issued
+            int s = 0;
+            uint32_t ph = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
                 Tile ti;
@@ -296,22 +396,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     continue;
                 const int n0 = ti.n0 * BN;
                 for (int kb = 0; kb < p.num_kb; ++kb) {
-                    // A scales of this K block into the scale ring
-                    if (!__all_sync(0xffffffffu, wait_one(bar_sempty + 8 * j, jph ^ 1, p, abort_flag))) {
-                        ok = false;
-                        break;
-                    }
-                    if (ptx::elect_one()) {
-                        ptx::mbar_arrive_expect_tx(bar_sfull + 8 * j, kSfaBytes);
-                        ptx::tma_load_3d(sfa_slot(j), &tmap_sfa, bar_sfull + 8 * j, ti.m0, kb, ti.a_z);
-                    }
-                    __syncwarp();
-                    ++n_sfa;
-                    if (++j == kSfaSlots) {
-                        j = 0;
-                        jph ^= 1;
-                    }
-                    // A and B tiles into the operand ring
                     if (!__all_sync(0xffffffffu, wait_one(bar_empty + 8 * s, ph ^ 1, p, abort_flag))) {
                         ok = false;
                         break;
@@ -330,24 +414,13 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     }
                 }
             }
-            // Wind down: every issued load must have landed before the CTA may exit.  In each
-            // ring only the last (ring size) loads can still be in flight; waiting on a slot's
-            // most recent phase returns at once if it was already consumed.
+            // Wind down: every issued load must have landed before the CTA may exit.  Only the
+            // last (ring size) loads can still be in flight; waiting on a slot's most recent
+            // phase returns at once if it was already consumed.
             {
-                int pending = n_sfa < static_cast<uint32_t>(kSfaSlots) ? static_cast<int>(n_sfa)
-                                                                        : kSfaSlots;
-                int dj = j;
-                uint32_t dph = jph;
-                for (int i = 0; i < pending; ++i) {
-                    if (--dj < 0) {
-                        dj = kSfaSlots - 1;
-                        dph ^= 1;
-                    }
-                    wait_drain(bar_sfull + 8 * dj, dph);
-                }
-                pending = n_op < static_cast<uint32_t>(p.stages) ? static_cast<int>(n_op) : p.stages;
+                int pending = n_op < static_cast<uint32_t>(p.stages) ? static_cast<int>(n_op) : p.stages;
                 int ds = s;
-                dph = ph;
+                uint32_t dph = ph;
                 for (int i = 0; i < pending; ++i) {
                     if (--ds < 0) {
                         ds = p.stages - 1;
@@ -418,8 +491,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                                    static_cast<uint32_t>(half * C::kCols);
         constexpr int P1 = C::kPart1;             // columns loaded before the first wait
         constexpr int P2 = C::kCols - P1;         // columns loaded after it (0 if all at once)
-        int j = 0;
-        uint32_t jph = 0;
         int buf = 0;
         uint32_t bph = 0;
         bool ok = true;
@@ -436,80 +507,24 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             const int split = min(C::kCols, max(0, (nb_lo + 1) * kBlockK - col0));  // first hi column
             const float *sfb_lo = p.sfb + (static_cast<size_t>(ti.g) * p.num_nb + nb_lo) * p.num_kb;
             const float *sfb_hi = p.sfb + (static_cast<size_t>(ti.g) * p.num_nb + nb_hi) * p.num_kb;
+            // this thread's A scales: one per K block, num_kb rows of sfa_ld apart (rows past the
+            // scale matrix read its last row; they are not stored)
+            const float *sa_ptr = p.sfa + static_cast<size_t>(ti.a_z) * p.num_kb * p.sfa_ld +
+                                  min(ti.m0 + row, p.sfa_ld - 1);
 
             float acc[C::kCols];
 #pragma unroll
             for (int c = 0; c < C::kCols; ++c)
                 acc[c] = 0.0f;
 
-            float sb_lo = __ldg(sfb_lo);
-            float sb_hi = __ldg(sfb_hi);
-            for (int kb = 0; kb < p.num_kb; ++kb) {
-                // prefetch the B scales of the next K block
-                const int kn = kb + 1 < p.num_kb ? kb + 1 : kb;
-                const float sb_lo_next = __ldg(sfb_lo + kn);
-                const float sb_hi_next = __ldg(sfb_hi + kn);
-                bool w = wait_one(bar_sfull + 8 * j, jph, p, abort_flag) &&
-                         wait_one(bar_tfull + 8 * buf, bph, p, abort_flag);
-                if (!__all_sync(0xffffffffu, w)) {
-                    ok = false;
-                    break;
-                }
-                ptx::tc_fence_after();
-                const uint32_t taddr = lane_base + static_cast<uint32_t>(buf * BN);
-                uint32_t pr[P1];
-                ptx::tmem_ld_cols<P1>(taddr, pr);
-                const float sa = sfa_ptr(j)[row];
-                const float scale_lo = sa * sb_lo;
-                const float scale_hi = sa * sb_hi;
-                ptx::tmem_wait_cols<P1>(pr);
-                if (P2 == 0) {
-                    // the whole partial is in registers: free the TMEM buffer and scale slot
-                    // before doing the arithmetic
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) {
-                        ptx::mbar_arrive(bar_tempty + 8 * buf);
-                        ptx::mbar_arrive(bar_sempty + 8 * j);
-                    }
-                }
-#pragma unroll
-                for (int g16 = 0; g16 < P1 / 16; ++g16) {
-                    const float sc = (16 * g16 >= split) ? scale_hi : scale_lo;
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        acc[16 * g16 + e] = fmaf(__uint_as_float(pr[16 * g16 + e]), sc, acc[16 * g16 + e]);
-                }
-                if (P2 > 0) {
-                    // second part reuses the same registers
-                    ptx::tmem_ld_cols<(P2 > 0 ? P2 : 16)>(taddr + P1, pr);
-                    ptx::tmem_wait_cols<(P2 > 0 ? P2 : 16)>(pr);
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) {
-                        ptx::mbar_arrive(bar_tempty + 8 * buf);
-                        ptx::mbar_arrive(bar_sempty + 8 * j);
-                    }
-#pragma unroll
-                    for (int g16 = 0; g16 < P2 / 16; ++g16) {
-                        const float sc = (P1 + 16 * g16 >= split) ? scale_hi : scale_lo;
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            acc[P1 + 16 * g16 + e] =
-                                fmaf(__uint_as_float(pr[16 * g16 + e]), sc, acc[P1 + 16 * g16 + e]);
-                    }
-                }
-                sb_lo = sb_lo_next;
-                sb_hi = sb_hi_next;
-                if (++j == kSfaSlots) {
-                    j = 0;
-                    jph ^= 1;
-                }
-                if (++buf == C::kTmemBufs) {
-                    buf = 0;
-                    bph ^= 1;
-                }
-            }
+            // scales of K blocks kb (cur) and kb + 1 (nxt) are in registers; kb + 2 is loaded
+            ok = promote_tile<BN, P1, P2, C::kCols, C::kTmemBufs>(
+                acc, sa_ptr, sfb_lo, sfb_hi, lane_base, bar_tfull, buf, bph,
+                [&](int b, uint32_t &rel, bool &remote) {
+                    rel = bar_tempty + 8 * b;
+                    remote = false;
+                },
+                split, lane, p, abort_flag);
             if (!ok)
                 break;
 

@@ -131,6 +131,13 @@ unsigned long long dg_set_wait_timeout_ns(unsigned long long ns);
  * Returns DG_ERR_INVALID_ARG for unsupported values. */
 int dg_set_config_override(int block_n, int num_stages);
 
+/* Tuning/testing switch between the two kernel families: 0 = automatic (default), 1 = always the
+ * one-CTA kernels, 2 = the CTA-pair kernels (tcgen05 cta_group::2, 256-row tiles) wherever the
+ * layout allows them (dense and masked; the contiguous layout always uses one-CTA tiles because
+ * its expert segments are only 128-row aligned).  Results are identical within the parity
+ * tolerance either way.  Returns the previous mode, or DG_ERR_INVALID_ARG. */
+int dg_set_pair_mode(int mode);
+
 /* Describes the most recent launch on this host thread: fills any non-NULL pointer with the
  * chosen block_n, pipeline stages, grid size (CTAs) and tile count.  Returns DG_OK, or
  * DG_ERR_INVALID_ARG when nothing was launched yet. */
