@@ -182,6 +182,22 @@ class ClockSampler:
                     reasons=sorted(self.reasons - {"gpu_idle"}), samples=len(self.samples))
 
 
+# ---- multi-rank aggregation ---------------------------------------------------------------------
+
+def max_over_ranks(seconds: float, world: int, device: str) -> float:
+    """The slowest rank's device time: every rank runs its own copy of the step (weak scaling),
+    so the job is done when the last rank is."""
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(flops_per_step: float, steps: int, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: the FLOPs all ranks did over the slowest rank's time."""
+    return world * flops_per_step * steps / max_seconds / 1e12
+
+
 # ---- our arm ------------------------------------------------------------------------------------
 
 class DeviceGemm:
@@ -228,8 +244,8 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     gemms, desc = build_workload(args.workload, args.shape)
-    if args.block_n or args.stages:
-        dg.set_config_override(args.block_n, args.stages)
+    if args.block_n or args.stages or args.splits:
+        dg.set_config_override(args.block_n, args.stages, args.splits)
     dev = [DeviceGemm(dg, g) for g in gemms]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
@@ -271,16 +287,13 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     total = sum(sum(p) for p in per)  # device seconds over the timed steps
-    t = torch.tensor([total], dtype=torch.float64, device="cuda")
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_max = float(t.item())
+    total_max = max_over_ranks(total, world, "cuda")
     if dg.poll_device_error(stream) != 0:
         raise RuntimeError("device error during the timed steps")
 
     flops_step = sum(g.flops for g in gemms)
     bytes_step = sum(g.bytes for g in gemms)
-    value = world * flops_step * args.steps / total_max / 1e12
+    value = aggregate_tflops(flops_step, args.steps, world, total_max)
     peaks = load_peaks()
     shapes = [roofline(g, statistics.mean(p), peaks) for g, p in zip(gemms, per)]
     dom = max(range(n), key=lambda i: sum(per[i]))
@@ -341,13 +354,11 @@ def run_e2e(dg, dev, gemms, args, world):
         step()
     steps = max(1, min(args.steps, 10))
     ts = [step() for _ in range(steps)]
-    t = torch.tensor([sum(ts)], dtype=torch.float64, device="cuda")
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    t_max = max_over_ranks(sum(ts), world, "cuda")
     flops = sum(g.flops for g in gemms)
-    return dict(value=world * flops * steps / float(t.item()) / 1e12, unit=UNIT,
+    return dict(value=aggregate_tflops(flops, steps, world, t_max), unit=UNIT,
                 h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, steps=steps,
-                ms_per_step=float(t.item()) / steps * 1e3)
+                ms_per_step=t_max / steps * 1e3)
 
 
 # ---- CPU oracle (baseline and reference arm) --------------------------------------------------
@@ -433,6 +444,7 @@ def main():
                     help="M,N,K of --workload dense")
     ap.add_argument("--block-n", type=int, default=0, help="tile override (tuning)")
     ap.add_argument("--stages", type=int, default=0, help="pipeline-stage override (tuning)")
+    ap.add_argument("--splits", type=int, default=0, help="split-K override (tuning)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

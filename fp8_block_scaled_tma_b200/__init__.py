@@ -67,12 +67,14 @@ def _load() -> ctypes.CDLL:
     lib.dg_poll_device_error.restype = i
     lib.dg_set_wait_timeout_ns.argtypes = [ctypes.c_ulonglong]
     lib.dg_set_wait_timeout_ns.restype = ctypes.c_ulonglong
-    lib.dg_set_config_override.argtypes = [i, i]
+    lib.dg_set_config_override.argtypes = [i, i, i]
     lib.dg_set_config_override.restype = i
-    lib.dg_set_pair_mode.argtypes = [i]
-    lib.dg_set_pair_mode.restype = i
+    lib.dg_set_fault_injection.argtypes = [i]
+    lib.dg_set_fault_injection.restype = i
+    lib.dg_set_kernel_family.argtypes = [i]
+    lib.dg_set_kernel_family.restype = i
     ipp = ctypes.POINTER(ctypes.c_int)
-    lib.dg_get_last_launch.argtypes = [ipp, ipp, ipp, ipp]
+    lib.dg_get_last_launch.argtypes = [ipp, ipp, ipp, ipp, ipp, ipp]
     lib.dg_get_last_launch.restype = i
     return lib
 
@@ -161,22 +163,37 @@ def set_wait_timeout_ns(ns: int) -> int:
     return int(lib.dg_set_wait_timeout_ns(int(ns)))
 
 
-def set_config_override(block_n: int = 0, num_stages: int = 0) -> None:
-    _check(lib.dg_set_config_override(int(block_n), int(num_stages)), "dg_set_config_override")
+def set_config_override(block_n: int = 0, num_stages: int = 0, splits: int = 0) -> None:
+    _check(lib.dg_set_config_override(int(block_n), int(num_stages), int(splits)),
+           "dg_set_config_override")
 
 
-def set_pair_mode(mode: int) -> int:
-    """0 automatic, 1 one-CTA kernels only, 2 CTA-pair kernels where the layout allows."""
-    r = lib.dg_set_pair_mode(int(mode))
+def set_fault_injection(mode: int) -> int:
+    """Test hook: 1 makes the MMA issuer wait on a barrier nothing signals (the watchdog then
+    reports DG_ERR_TIMEOUT); 0 turns it off.  Returns the previous mode."""
+    r = lib.dg_set_fault_injection(int(mode))
     if r < 0:
-        raise DGError(r, "dg_set_pair_mode")
+        raise DGError(r, "dg_set_fault_injection")
+    return r
+
+
+FAMILY_AUTO, FAMILY_ONE_CTA, FAMILY_PAIR, FAMILY_SPLIT_K = 0, 1, 2, 3
+
+
+def set_kernel_family(family: int) -> int:
+    """0 automatic, 1 one-CTA kernels, 2 CTA-pair kernels where the layout allows, 3 split-K
+    cluster kernel for dense calls.  Returns the previous value."""
+    r = lib.dg_set_kernel_family(int(family))
+    if r < 0:
+        raise DGError(r, "dg_set_kernel_family")
     return r
 
 
 def get_last_launch() -> dict:
-    v = [ctypes.c_int() for _ in range(4)]
+    v = [ctypes.c_int() for _ in range(6)]
     _check(lib.dg_get_last_launch(*[ctypes.byref(x) for x in v]), "dg_get_last_launch")
-    return dict(block_n=v[0].value, stages=v[1].value, grid=v[2].value, tiles=v[3].value)
+    return dict(block_n=v[0].value, stages=v[1].value, grid=v[2].value, tiles=v[3].value,
+                family=v[4].value, splits=v[5].value)
 
 
 def sfa_mn_major(sa: torch.Tensor) -> torch.Tensor:

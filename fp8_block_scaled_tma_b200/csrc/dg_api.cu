@@ -13,6 +13,7 @@
 #include "../../include/dg.h"
 #include "dg_kernel.cuh"
 #include "dg_pair_kernel.cuh"
+#include "dg_splitk_kernel.cuh"
 
 namespace {
 
@@ -40,16 +41,22 @@ struct KernelSmem {
 };
 KernelSmem g_smem[kMaxDevices][3][8];       // 1-CTA kernels, per device / layout / BN
 KernelSmem g_smem_pair[kMaxDevices][3][8];  // CTA-pair kernels
-int g_pair_mode = 0;                        // 0 auto, 1 single-CTA kernels only, 2 pairs where possible
+KernelSmem g_smem_split[kMaxDevices][8];    // split-K kernels, per BN
+int g_family = 0;  // 0 auto, 1 one-CTA kernels, 2 CTA pairs where possible, 3 split-K (dense)
 int g_num_sms_cap = 0;
 unsigned long long g_timeout_ns = kDefaultTimeoutNs;
 int g_override_bn = 0;
 int g_override_stages = 0;
+int g_override_splits = 0;
+int g_inject_stall = 0;
+// clusters of each size (index = cluster size, 1..8) that can be resident at once, per device
+// and kernel family; 0 = not queried yet
+int g_max_clusters[kMaxDevices][3][9];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 struct LastLaunch {
     bool valid = false;
-    int block_n = 0, stages = 0, grid = 0, tiles = 0, pair = 0;
+    int block_n = 0, stages = 0, grid = 0, tiles = 0, pair = 0, splits = 1, family = 1;
 };
 thread_local LastLaunch t_last;
 
@@ -113,6 +120,12 @@ int device_setup(int &dev_out, DeviceInfo *&info)
     dev_out = dev;
     info = &d;
     return d.status;
+}
+
+int inject_stall_flag()
+{
+    std::lock_guard<std::mutex> lock(g_mutex);
+    return g_inject_stall;
 }
 
 bool aligned16(const void *p)
@@ -217,6 +230,101 @@ int choose_pair_block_n(long long pair_row_tiles, int N, int num_pairs)
     return best_bn;
 }
 
+template <int BN>
+void *splitk_kernel_ptr()
+{
+    return reinterpret_cast<void *>(&dg::dg_gemm_splitk_kernel<BN>);
+}
+
+void *pick_splitk_kernel(int bn)
+{
+    switch (bn) {
+    case 64: return splitk_kernel_ptr<64>();
+    case 96: return splitk_kernel_ptr<96>();
+    case 128: return splitk_kernel_ptr<128>();
+    case 160: return splitk_kernel_ptr<160>();
+    case 192: return splitk_kernel_ptr<192>();
+    case 224: return splitk_kernel_ptr<224>();
+    case 256: return splitk_kernel_ptr<256>();
+    default: return nullptr;
+    }
+}
+
+// Largest number of clusters of `csize` CTAs (one CTA per SM, `dyn_smem` bytes each) that can be
+// resident at once: clusters live inside one GPC, so this can be below sms / csize.
+int max_active_clusters(void *fn, int csize, int dyn_smem, int dev, int family_slot)
+{
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        int v = g_max_clusters[dev][family_slot][csize];
+        if (v > 0)
+            return v;
+    }
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(csize, 1, 1);
+    cfg.blockDim = dim3(dg::kNumThreads, 1, 1);
+    cfg.dynamicSmemBytes = dyn_smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return 0;
+    }
+    std::lock_guard<std::mutex> lock(g_mutex);
+    g_max_clusters[dev][family_slot][csize] = n;
+    return n;
+}
+
+// Split-K choice for dense problems with few output tiles: BN and the number of K splits S
+// (cluster size) minimising a simple time model -- the larger of the per-CTA TMA time (bytes
+// the CTA copies at ~100 GB/s), the whole problem's HBM time and the per-CTA MMA issue time --
+// plus a fixed launch/prologue cost and the cross-CTA reduction.  Returns false if no
+// configuration fits in one wave of CTAs.
+template <class Capacity>
+bool choose_splitk(int M, int N, int K, int sms, int bn_fixed, int s_fixed, Capacity capacity,
+                   int &bn_out, int &s_out)
+{
+    const int num_kb = K / dg::kBlockK;
+    const int m_tiles = (M + dg::kBlockM - 1) / dg::kBlockM;
+    double best = 1e300;
+    bool found = false;
+    for (int bn = 256; bn >= 64; bn -= 32) {
+        if (bn_fixed != 0 && bn != bn_fixed)
+            continue;
+        const long long tiles = static_cast<long long>(m_tiles) * ((N + bn - 1) / bn);
+        if (tiles > sms)
+            continue;
+        const int s_max = static_cast<int>(std::min<long long>(std::min(dg::kMaxSplits, num_kb), sms / tiles));
+        for (int S = 1; S <= s_max; ++S) {
+            if (s_fixed != 0 && S != s_fixed)
+                continue;
+            // every cluster of the grid must be resident at once (one wave)
+            if (tiles > capacity(bn, S))
+                continue;
+            const int kb_per = (num_kb + S - 1) / S;
+            const double t_tma = kb_per * (16384.0 + bn * 128.0) / 100.0;                 // ns
+            const double t_hbm = (static_cast<double>(N) * K + static_cast<double>(M) * K) / 6500.0;
+            const double t_mma = kb_per * std::max(2.0 * bn, 230.0) / 1.9;
+            const double t_red = S > 1 ? 300.0 + 100.0 * S : 0.0;
+            const double t = std::max(t_tma, std::max(t_hbm, t_mma)) + 1500.0 + t_red;
+            if (t < best - 1e-9) {
+                best = t;
+                bn_out = bn;
+                s_out = S;
+                found = true;
+            }
+        }
+    }
+    return found;
+}
+
 template <int L, int BN>
 void *kernel_ptr()
 {
@@ -284,6 +392,116 @@ struct LaunchArgs {
     int expected_m;
     void *stream;
 };
+
+int launch_splitk(const LaunchArgs &args, int dev, DeviceInfo *info, int bn, int S,
+                  int stages_override, unsigned long long timeout)
+{
+    const int M = args.M, N = args.N, K = args.K;
+    const int num_kb = K / dg::kBlockK;
+    const int num_nb = (N + dg::kBlockK - 1) / dg::kBlockK;
+    const int m_tiles = (M + dg::kBlockM - 1) / dg::kBlockM;
+    const int n_tiles = (N + bn - 1) / bn;
+    void *fn = pick_splitk_kernel(bn);
+    if (fn == nullptr)
+        return DG_ERR_INVALID_ARG;
+    const int sbytes = dg::kSplitKbPerStage * (dg::kBlockM * dg::kBlockK + bn * dg::kBlockK);
+    const int part_bytes = dg::kBlockM * (bn + 4) * 4;
+    int stages = 0, dyn_smem = 0;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        KernelSmem &ks = g_smem_split[dev][bn / 32 - 1];
+        if (ks.static_bytes < 0) {
+            cudaFuncAttributes fa;
+            cudaError_t e = cudaFuncGetAttributes(&fa, fn);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                return DG_ERR_CUDA;
+            }
+            ks.static_bytes = static_cast<int>(fa.sharedSizeBytes);
+        }
+        const int dyn_cap = info->smem_optin - ks.static_bytes;
+        stages = std::min(dg::kMaxStages, (dyn_cap - 1024) / sbytes);
+        if (stages_override > 0)
+            stages = std::min(stages, stages_override);
+        if (stages < 2 || part_bytes + 1024 > dyn_cap)
+            return DG_ERR_UNSUPPORTED;
+        // the pipeline buffers, reused for the fp32 partial tile after the K loop
+        dyn_smem = std::max(stages * sbytes, part_bytes) + 1024;
+        dyn_smem = std::min(std::max(dyn_smem, kMinDynSmem), dyn_cap);
+        if (ks.limit_set < dyn_smem) {
+            cudaError_t e =
+                cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                return DG_ERR_CUDA;
+            }
+            ks.limit_set = dyn_smem;
+        }
+    }
+    CUtensorMap map_a, map_b;
+    if (make_map_kblocks(&map_a, const_cast<void *>(args.a), K, M, 1, dg::kBlockM,
+                         dg::kSplitKbPerStage) != DG_OK ||
+        make_map_kblocks(&map_b, const_cast<void *>(args.b), K, N, 1, bn, dg::kSplitKbPerStage) !=
+            DG_OK) {
+        if (debug_enabled())
+            std::fprintf(stderr, "[dg] cuTensorMapEncodeTiled failed (split-K)\n");
+        return DG_ERR_CUDA;
+    }
+    Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.G = 1;
+    p.num_kb = num_kb;
+    p.num_nb = num_nb;
+    p.m_tiles = m_tiles;
+    p.n_tiles = n_tiles;
+    p.stages = stages;
+    p.raster_m = S;
+    p.sfa = args.sfa;
+    p.sfa_ld = align4(M);
+    p.sfb = args.sfb;
+    p.d = static_cast<__nv_bfloat16 *>(args.d);
+    p.err = info->err_ptr;
+    p.timeout_ns = timeout;
+    p.inject_stall = inject_stall_flag();
+    p.num_tiles = m_tiles * n_tiles;
+
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(p.num_tiles * S, 1, 1);
+    cfg.blockDim = dim3(dg::kNumThreads, 1, 1);
+    cfg.dynamicSmemBytes = dyn_smem;
+    cfg.stream = static_cast<cudaStream_t>(args.stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void *kargs[] = {&map_a, &map_b, &p};
+    cudaError_t e = cudaLaunchKernelExC(&cfg, fn, kargs);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        if (debug_enabled())
+            std::fprintf(stderr, "[dg] split-K launch failed: %s\n", cudaGetErrorString(e));
+        return DG_ERR_CUDA;
+    }
+    t_last.valid = true;
+    t_last.block_n = bn;
+    t_last.stages = stages;
+    t_last.grid = p.num_tiles * S;
+    t_last.tiles = p.num_tiles;
+    t_last.pair = 0;
+    t_last.splits = S;
+    t_last.family = 3;
+    if (debug_enabled())
+        std::fprintf(stderr, "[dg] split-K M=%d N=%d K=%d BN=%d S=%d stages=%d grid=%d smem=%d\n", M, N,
+                     K, bn, S, stages, p.num_tiles * S, dyn_smem);
+    return DG_OK;
+}
 
 int launch_pair(const LaunchArgs &args, int dev, DeviceInfo *info, int sms, int bn,
                 int stages_override, unsigned long long timeout)
@@ -377,13 +595,17 @@ int launch_pair(const LaunchArgs &args, int dev, DeviceInfo *info, int sms, int 
     p.masked_m = args.masked_m;
     p.err = info->err_ptr;
     p.timeout_ns = timeout;
+    p.inject_stall = inject_stall_flag();
     long long tiles = (args.layout == dg::kMasked)
                           ? static_cast<long long>(G) * pair_m_tiles * n_tiles
                           : static_cast<long long>(pair_m_tiles) * n_tiles;
     if (tiles > 0x7FFFFFFFLL)
         return DG_ERR_INVALID_ARG;
     p.num_tiles = static_cast<int>(tiles);
-    const int pairs = static_cast<int>(std::min<long long>(num_pairs, tiles));
+    int resident = max_active_clusters(fn, 2, dyn_smem, dev, args.layout == dg::kDense ? 0 : 1);
+    if (resident <= 0 || resident > num_pairs)
+        resident = num_pairs;
+    const int pairs = static_cast<int>(std::min<long long>(resident, tiles));
     if (pairs <= 0)
         return DG_OK;
 
@@ -414,6 +636,8 @@ int launch_pair(const LaunchArgs &args, int dev, DeviceInfo *info, int sms, int 
     t_last.grid = 2 * pairs;
     t_last.tiles = p.num_tiles;
     t_last.pair = 1;
+    t_last.splits = 1;
+    t_last.family = 2;
     if (debug_enabled())
         std::fprintf(stderr, "[dg] pair layout=%d M=%d N=%d K=%d G=%d BN=%d stages=%d grid=%d tiles=%d smem=%d\n",
                      args.layout, M, N, K, G, bn, stages, 2 * pairs, p.num_tiles, dyn_smem);
@@ -449,12 +673,34 @@ int launch(const LaunchArgs &args)
         bn = g_override_bn;
         stages_override = g_override_stages;
         timeout = g_timeout_ns;
-        pair_mode = g_pair_mode;
+        pair_mode = g_family;
+    }
+    // Split-K clusters for dense problems with few output tiles (the memory-bound small-M
+    // regime): auto mode uses them for M <= 256.
+    if (args.layout == dg::kDense && (pair_mode == 3 || (pair_mode == 0 && M <= 256)) &&
+        (bn == 0 || pick_splitk_kernel(bn) != nullptr)) {
+        int sbn = 0, S = 0;
+        int splits_override;
+        {
+            std::lock_guard<std::mutex> lock(g_mutex);
+            splits_override = g_override_splits;
+        }
+        auto capacity = [&](int cbn, int cs) -> long long {
+            void *fn = pick_splitk_kernel(cbn);
+            const int sb = dg::kSplitKbPerStage * (dg::kBlockM * dg::kBlockK + cbn * dg::kBlockK);
+            const int smem = std::max(std::min(2 * sb, 200 * 1024), kMinDynSmem);
+            int n = max_active_clusters(fn, cs, smem, dev, 2);
+            if (n <= 0)
+                n = sms / cs;
+            return std::min<long long>(n, sms / cs);
+        };
+        if (choose_splitk(M, N, K, sms, bn, splits_override, capacity, sbn, S))
+            return launch_splitk(args, dev, info, sbn, S, stages_override, timeout);
     }
     // CTA pairs (cta_group::2) for the dense and masked layouts: 256-row tiles whose B half is
     // loaded by each CTA.  Auto mode uses them when a tile of 256 rows is mostly useful.
     bool use_pair = false;
-    if (args.layout != dg::kContiguous && sms >= 2 && pair_mode != 1) {
+    if (args.layout != dg::kContiguous && sms >= 2 && pair_mode != 1 && pair_mode != 3) {
         if (pair_mode == 2)
             use_pair = true;
         else if (args.layout == dg::kDense)
@@ -556,6 +802,7 @@ int launch(const LaunchArgs &args)
     p.masked_m = args.masked_m;
     p.err = info->err_ptr;
     p.timeout_ns = timeout;
+    p.inject_stall = inject_stall_flag();
     long long tiles;
     if (args.layout == dg::kMasked)
         tiles = static_cast<long long>(G) * m_tiles * n_tiles;  // upper bound; exact on device
@@ -590,6 +837,8 @@ int launch(const LaunchArgs &args)
     t_last.grid = grid;
     t_last.tiles = p.num_tiles;
     t_last.pair = 0;
+    t_last.splits = 1;
+    t_last.family = 1;
     if (debug_enabled())
         std::fprintf(stderr, "[dg] layout=%d M=%d N=%d K=%d G=%d BN=%d stages=%d grid=%d tiles=%d smem=%d\n",
                      args.layout, M, N, K, G, bn, stages, grid, p.num_tiles, dyn_smem);
@@ -769,32 +1018,50 @@ unsigned long long dg_set_wait_timeout_ns(unsigned long long ns)
     return prev;
 }
 
-int dg_set_config_override(int block_n, int num_stages)
+int dg_set_config_override(int block_n, int num_stages, int splits)
 {
     if (block_n != 0 && (block_n < 32 || block_n > 256 || block_n % 32 != 0))
         return DG_ERR_INVALID_ARG;
     if (num_stages != 0 && (num_stages < 2 || num_stages > dg::kMaxStages))
         return DG_ERR_INVALID_ARG;
+    if (splits < 0 || splits > dg::kMaxSplits)
+        return DG_ERR_INVALID_ARG;
     std::lock_guard<std::mutex> lock(g_mutex);
     g_override_bn = block_n;
     g_override_stages = num_stages;
+    g_override_splits = splits;
     return DG_OK;
 }
 
-int dg_set_pair_mode(int mode)
+int dg_set_fault_injection(int mode)
 {
-    if (mode < 0 || mode > 2)
+    if (mode < 0 || mode > 1)
         return DG_ERR_INVALID_ARG;
     std::lock_guard<std::mutex> lock(g_mutex);
-    int prev = g_pair_mode;
-    g_pair_mode = mode;
+    int prev = g_inject_stall;
+    g_inject_stall = mode;
     return prev;
 }
 
-int dg_get_last_launch(int *block_n, int *num_stages, int *grid, int *num_tiles)
+int dg_set_kernel_family(int family)
+{
+    if (family < 0 || family > 3)
+        return DG_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int prev = g_family;
+    g_family = family;
+    return prev;
+}
+
+int dg_get_last_launch(int *block_n, int *num_stages, int *grid, int *num_tiles, int *family,
+                       int *splits)
 {
     if (!t_last.valid)
         return DG_ERR_INVALID_ARG;
+    if (family)
+        *family = t_last.family;
+    if (splits)
+        *splits = t_last.splits;
     if (block_n)
         *block_n = t_last.block_n;
     if (num_stages)

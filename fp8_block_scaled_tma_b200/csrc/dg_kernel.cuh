@@ -68,6 +68,7 @@ struct Params {
     const int *masked_m;
     int *err;
     unsigned long long timeout_ns;
+    int inject_stall;   // test hook: the MMA issuer first waits on a barrier nothing signals
 };
 
 template <int BN>
@@ -96,6 +97,7 @@ struct SmemCtl {
     uint64_t tmem_full[4];
     uint64_t tmem_empty[4];
     uint64_t drain;
+    uint64_t stall;      // never signalled: the target of the fault-injection test hook
     uint32_t tmem_base;
     int abort_flag;
     int total_tiles;
@@ -347,6 +349,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             ptx::mbar_init(bar_tempty + 8 * b, kNumMathWarps);
         }
         ptx::mbar_init(bar_drain, 1);
+        ptx::mbar_init(ptx::smem_addr(&ctl.stall), 1);
         ctl.abort_flag = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tmap_a);
@@ -436,7 +439,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             uint32_t ph = 0;
             int buf = 0;
             uint32_t bph = 0;
-            bool ok = true;
+            bool ok = !p.inject_stall ||
+                      __all_sync(0xffffffffu, wait_one(ptx::smem_addr(&ctl.stall), 0, p, abort_flag));
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
                 Tile ti;
                 if (!resolve_tile<L>(p, ctl, t, ti))

@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             ptx::mbar_init(bar_tempty + 8 * b, 2 * kNumMathWarps); // both CTAs' promotion warps
         }
         ptx::mbar_init(bar_drain, 1);
+        ptx::mbar_init(ptx::smem_addr(&ctl.stall), 1);
         ctl.abort_flag = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tmap_a);
@@ -277,7 +278,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             uint32_t ph = 0;
             int buf = 0;
             uint32_t bph = 0;
-            bool ok = true;
+            bool ok = !p.inject_stall ||
+                      __all_sync(0xffffffffu, wait_one_c(ptx::smem_addr(&ctl.stall), 0, p, abort_flag));
             for (int t = pair; t < num_tiles && ok; t += num_pairs) {
                 for (int kb0 = 0; kb0 < p.num_kb && ok; kb0 += KS) {
                     if (!__all_sync(0xffffffffu, wait_one_c(bar_full + 8 * s, ph, p, abort_flag))) {

@@ -126,22 +126,35 @@ int dg_poll_device_error(void *stream);
  * hanging.  0 restores the default.  Returns the previous value. */
 unsigned long long dg_set_wait_timeout_ns(unsigned long long ns);
 
-/* Tuning/testing override of the tile choice: block_n in {32, 64, ..., 256} (the N extent of a
- * tile; 0 = heuristic) and the number of shared-memory pipeline stages (0 = as many as fit).
- * Returns DG_ERR_INVALID_ARG for unsupported values. */
-int dg_set_config_override(int block_n, int num_stages);
+/* Test hook for the watchdog: mode 1 makes every following launch's MMA issuer first wait on a
+ * barrier that nothing signals, so the wait runs out after the dg_set_wait_timeout_ns limit and
+ * the kernel reports DG_ERR_TIMEOUT and winds down (no fault, no hang).  0 (default) turns it
+ * off.  Returns the previous mode, or DG_ERR_INVALID_ARG. */
+int dg_set_fault_injection(int mode);
 
-/* Tuning/testing switch between the two kernel families: 0 = automatic (default), 1 = always the
- * one-CTA kernels, 2 = the CTA-pair kernels (tcgen05 cta_group::2, 256-row tiles) wherever the
+/* Tuning/testing override of the tile choice: block_n in {32, 64, ..., 256} (the N extent of a
+ * tile; 0 = heuristic), the number of shared-memory pipeline stages (0 = as many as fit) and the
+ * number of K splits of the split-K kernel (1..8; 0 = heuristic).  Returns DG_ERR_INVALID_ARG
+ * for unsupported values. */
+int dg_set_config_override(int block_n, int num_stages, int splits);
+
+/* Tuning/testing switch between the kernel families: 0 = automatic (default); 1 = the one-CTA
+ * persistent kernels; 2 = the CTA-pair kernels (tcgen05 cta_group::2, 256-row tiles) wherever the
  * layout allows them (dense and masked; the contiguous layout always uses one-CTA tiles because
- * its expert segments are only 128-row aligned).  Results are identical within the parity
- * tolerance either way.  Returns the previous mode, or DG_ERR_INVALID_ARG. */
-int dg_set_pair_mode(int mode);
+ * its expert segments are only 128-row aligned); 3 = the split-K cluster kernel for dense calls
+ * whose output tiles fit in one wave (the K blocks of a tile are split over up to 8 CTAs that
+ * reduce their fp32 partials through distributed shared memory, in a fixed order).  Automatic
+ * mode uses split-K for dense M <= 256, pairs for larger dense M and for masked calls.  Results
+ * agree within the parity tolerance whichever family runs.  Returns the previous value, or
+ * DG_ERR_INVALID_ARG. */
+int dg_set_kernel_family(int family);
 
 /* Describes the most recent launch on this host thread: fills any non-NULL pointer with the
- * chosen block_n, pipeline stages, grid size (CTAs) and tile count.  Returns DG_OK, or
- * DG_ERR_INVALID_ARG when nothing was launched yet. */
-int dg_get_last_launch(int *block_n, int *num_stages, int *grid, int *num_tiles);
+ * chosen block_n, pipeline stages, grid size (CTAs), output tile count, kernel family (1, 2 or
+ * 3 as in dg_set_kernel_family) and K splits per tile.  Returns DG_OK, or DG_ERR_INVALID_ARG
+ * when nothing was launched yet. */
+int dg_get_last_launch(int *block_n, int *num_stages, int *grid, int *num_tiles, int *family,
+                       int *splits);
 
 #ifdef __cplusplus
 }

@@ -68,11 +68,16 @@ def test_num_sms_cap_roundtrip(dg):
 
 
 def test_config_override_validation(dg):
-    assert dg.lib.dg_set_config_override(100, 0) == dg.DG_ERR_INVALID_ARG
-    assert dg.lib.dg_set_config_override(0, 1) == dg.DG_ERR_INVALID_ARG
-    assert dg.lib.dg_set_config_override(0, 9) == dg.DG_ERR_INVALID_ARG
-    assert dg.lib.dg_set_config_override(96, 4) == dg.DG_OK
-    assert dg.lib.dg_set_config_override(0, 0) == dg.DG_OK
+    assert dg.lib.dg_set_config_override(100, 0, 0) == dg.DG_ERR_INVALID_ARG
+    assert dg.lib.dg_set_config_override(0, 1, 0) == dg.DG_ERR_INVALID_ARG
+    assert dg.lib.dg_set_config_override(0, 9, 0) == dg.DG_ERR_INVALID_ARG
+    assert dg.lib.dg_set_config_override(0, 0, 9) == dg.DG_ERR_INVALID_ARG
+    assert dg.lib.dg_set_config_override(96, 4, 3) == dg.DG_OK
+    assert dg.lib.dg_set_config_override(0, 0, 0) == dg.DG_OK
+    assert dg.lib.dg_set_kernel_family(4) == dg.DG_ERR_INVALID_ARG
+    assert dg.lib.dg_set_fault_injection(2) == dg.DG_ERR_INVALID_ARG
+    assert dg.lib.dg_set_fault_injection(0) == dg.DG_OK
+    assert dg.lib.dg_set_kernel_family(0) == dg.DG_OK
 
 
 def test_timeout_setter(dg):
