@@ -153,13 +153,26 @@ int make_map(CUtensorMap *map, CUtensorMapDataType dt, void *base, uint64_t d0, 
     return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
 }
 
+// 2-D view [rows][N] of the bf16 output for the TMA-store epilogue: one box is 32 rows x 16
+// columns (32-byte rows, 32-byte swizzle), matching the kernels' staging boxes.
+int make_map_d(CUtensorMap *map, void *base, uint64_t N, uint64_t rows)
+{
+    cuuint64_t dims[2] = {N, rows};
+    cuuint64_t strides[1] = {N * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(dg::kEpiCols), static_cast<cuuint32_t>(dg::kEpiRows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
+}
+
 int stage_bytes_rt(int bn)
 {
     return dg::kBlockM * dg::kBlockK + bn * dg::kBlockK;  // A tile + B tile (multiple of 1024)
 }
 
 
-using KernelFn = void (*)(CUtensorMap, CUtensorMap, Params);
 
 // 4-D view [groups][K/128][rows][128 bytes] of a K-major uint8 operand: one box holds `kbs`
 // consecutive 128-wide K blocks of `box_rows` rows, laid out K block by K block in shared memory.
@@ -210,18 +223,32 @@ int pair_stage_bytes(int bn)
 constexpr int kPairSfaRingBytes = dg::kSfaSlots * dg::kKbPerStage * dg::kBlockM * 4;
 
 // Tile heuristic of the pair kernel: 256-row pair tiles, waves over SM pairs.
+// Time model shared by the tile choosers.  A persistent CTA (or CTA pair) walks its tiles one
+// after another, so the time is (tiles per CTA, rounded up) x (time of one tile).  Measured on
+// B200 (dense 4096-row shapes, every BN from 128 to 256, both kernel families), one K block of
+// one 128-row tile costs about kTileFixed + BN column-units: a fixed part (the MMA-commit ->
+// promotion -> buffer-release round trip) plus a part proportional to the tile width (MMA,
+// tensor-memory reads and FFMA promotion).  Columns computed past N are wasted work.
+constexpr double kTileFixed = 190.0;
+// Dense problems use CTA pairs only for long K: measured on B200, the pair kernel is ahead by a
+// few percent at K = 16384 and level with or behind the one-CTA kernel at K <= 7168, where its
+// longer per-tile start-up weighs more.
+constexpr int kPairMinKBlocks = 96;
+
+double tile_time(long long row_tiles, int N, int bn, int slots)
+{
+    const long long n_tiles = (N + bn - 1) / bn;
+    const long long tiles = n_tiles * row_tiles;
+    const long long waves = (tiles + slots - 1) / slots;
+    return static_cast<double>(waves) * (kTileFixed + bn);
+}
+
 int choose_pair_block_n(long long pair_row_tiles, int N, int num_pairs)
 {
     int best_bn = 256;
     double best = 1e300;
     for (int bn = 128; bn <= 256; bn += 32) {
-        long long n_tiles = (N + bn - 1) / bn;
-        long long tiles = n_tiles * pair_row_tiles;
-        long long waves = (tiles + num_pairs - 1) / num_pairs;
-        double per_tile = static_cast<double>(bn) + 16.0;
-        double t = waves * per_tile;
-        double waste = static_cast<double>(n_tiles * bn - N) / N;
-        t *= 1.0 + 0.5 * waste;
+        const double t = tile_time(pair_row_tiles, N, bn, num_pairs);
         if (t < best - 1e-9 || (std::abs(t - best) <= 1e-9 && bn > best_bn)) {
             best = t;
             best_bn = bn;
@@ -356,20 +383,12 @@ void *pick_kernel(int layout, int bn)
 // Tile heuristic: among BN in {32..256} pick the one with the smallest estimated time, where a
 // tile of BN columns costs max(MMA time ~ BN, load time ~ 128 + BN) and tiles run in waves over
 // the SMs (non-power-of-two BN exists to even out the last wave).
-int choose_block_n(int rows_tiles, int N, int num_sms, long long expected_rows_total)
+int choose_block_n(int rows_tiles, int N, int num_sms)
 {
-    (void)expected_rows_total;
-    int best_bn = 128;
+    int best_bn = 256;
     double best = 1e300;
     for (int bn = 32; bn <= 256; bn += 32) {
-        long long n_tiles = (N + bn - 1) / bn;
-        long long tiles = n_tiles * rows_tiles;
-        long long waves = (tiles + num_sms - 1) / num_sms;
-        double per_tile = std::max(static_cast<double>(bn), 0.55 * (128.0 + bn)) + 24.0;
-        double t = waves * per_tile;
-        // avoid wasting columns past N
-        double waste = static_cast<double>(n_tiles * bn - N) / N;
-        t *= 1.0 + 0.5 * waste;
+        const double t = tile_time(rows_tiles, N, bn, num_sms);
         if (t < best - 1e-9 || (std::abs(t - best) <= 1e-9 && bn > best_bn)) {
             best = t;
             best_bn = bn;
@@ -538,13 +557,14 @@ int launch_pair(const LaunchArgs &args, int dev, DeviceInfo *info, int sms, int 
             ks.static_bytes = static_cast<int>(fa.sharedSizeBytes);
         }
         const int dyn_cap = info->smem_optin - ks.static_bytes;
-        stages = std::min(dg::kMaxStages, (dyn_cap - 1024 - kPairSfaRingBytes) / sbytes);
+        stages = std::min(dg::kMaxStages, (dyn_cap - 1024 - kPairSfaRingBytes - dg::kEpiBytes) / sbytes);
         if (stages_override > 0)
             stages = std::min(stages, stages_override);
         if (stages < 2)
             return DG_ERR_UNSUPPORTED;
-        // operand stages, the A-scale ring, and slack to align the stages to 1024 bytes
-        dyn_smem = stages * sbytes + kPairSfaRingBytes + 1024;
+        // operand stages, the A-scale ring, the output staging boxes, and slack to align the
+        // stages to 1024 bytes
+        dyn_smem = stages * sbytes + kPairSfaRingBytes + dg::kEpiBytes + 1024;
         dyn_smem = std::min(std::max(dyn_smem, kMinDynSmem), dyn_cap);
         if (ks.limit_set < dyn_smem) {
             cudaError_t e =
@@ -560,8 +580,9 @@ int launch_pair(const LaunchArgs &args, int dev, DeviceInfo *info, int sms, int 
     const int a_groups = (args.layout == dg::kMasked) ? G : 1;
     const int b_groups = (args.layout == dg::kDense) ? 1 : G;
     const int m4 = align4(M);
-    CUtensorMap map_a, map_b, map_sfa;
-    if (make_map_kblocks(&map_a, const_cast<void *>(args.a), K, M, a_groups, dg::kBlockM,
+    CUtensorMap map_a, map_b, map_sfa, map_d;
+    if (make_map_d(&map_d, args.d, N, static_cast<uint64_t>(M) * a_groups) != DG_OK ||
+        make_map_kblocks(&map_a, const_cast<void *>(args.a), K, M, a_groups, dg::kBlockM,
                          dg::kKbPerStage) != DG_OK ||
         make_map_kblocks(&map_b, const_cast<void *>(args.b), K, N, b_groups, bn / 2,
                          dg::kKbPerStage) != DG_OK ||
@@ -622,7 +643,7 @@ int launch_pair(const LaunchArgs &args, int dev, DeviceInfo *info, int sms, int 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    void *kargs[] = {&map_a, &map_b, &map_sfa, &p};
+    void *kargs[] = {&map_a, &map_b, &map_sfa, &map_d, &p};
     cudaError_t e = cudaLaunchKernelExC(&cfg, fn, kargs);
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -698,13 +719,14 @@ int launch(const LaunchArgs &args)
             return launch_splitk(args, dev, info, sbn, S, stages_override, timeout);
     }
     // CTA pairs (cta_group::2) for the dense and masked layouts: 256-row tiles whose B half is
-    // loaded by each CTA.  Auto mode uses them when a tile of 256 rows is mostly useful.
+    // loaded by each CTA.  Auto mode uses them when a tile of 256 rows is mostly useful and, for
+    // dense problems, K is long (kPairMinKBlocks).
     bool use_pair = false;
     if (args.layout != dg::kContiguous && sms >= 2 && pair_mode != 1 && pair_mode != 3) {
         if (pair_mode == 2)
             use_pair = true;
         else if (args.layout == dg::kDense)
-            use_pair = M > 192;
+            use_pair = M > 192 && num_kb >= kPairMinKBlocks;
         else
             use_pair = args.expected_m == 0 || args.expected_m > 64;
         if (bn != 0 && pick_pair_kernel(args.layout, bn) == nullptr)
@@ -718,7 +740,7 @@ int launch(const LaunchArgs &args)
             int em = args.expected_m > 0 ? std::min(args.expected_m, M) : M;
             row_tiles = static_cast<long long>(G) * ((em + dg::kBlockM - 1) / dg::kBlockM);
         }
-        bn = choose_block_n(static_cast<int>(std::max<long long>(1, row_tiles)), N, sms, 0);
+        bn = choose_block_n(static_cast<int>(std::max<long long>(1, row_tiles)), N, sms);
     }
     const int n_tiles = (N + bn - 1) / bn;
     const int sbytes = stage_bytes_rt(bn);
@@ -744,12 +766,13 @@ int launch(const LaunchArgs &args)
             ks.static_bytes = static_cast<int>(fa.sharedSizeBytes);
         }
         const int dyn_cap = info->smem_optin - ks.static_bytes;  // dynamic bytes allowed
-        stages = std::min(dg::kMaxStages, (dyn_cap - 1024) / sbytes);
+        stages = std::min(dg::kMaxStages, (dyn_cap - 1024 - dg::kEpiBytes) / sbytes);
         if (stages_override > 0)
             stages = std::min(stages, stages_override);
         if (stages < 2)
             return DG_ERR_UNSUPPORTED;
-        dyn_smem = stages * sbytes + 1024;  // + slack to align the stages to 1024 bytes
+        // operand stages, the output staging boxes, and slack to align the stages to 1024 bytes
+        dyn_smem = stages * sbytes + dg::kEpiBytes + 1024;
         dyn_smem = std::min(std::max(dyn_smem, kMinDynSmem), dyn_cap);
         if (ks.limit_set < dyn_smem) {
             cudaError_t e =
@@ -770,8 +793,9 @@ int launch(const LaunchArgs &args)
     const int a_groups = (args.layout == dg::kMasked) ? G : 1;
     const int b_groups = (args.layout == dg::kDense) ? 1 : G;
     const int m4 = align4(M);
-    CUtensorMap map_a, map_b;
-    if (make_map(&map_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<void *>(args.a), K, a_rows,
+    CUtensorMap map_a, map_b, map_d;
+    if (make_map_d(&map_d, args.d, N, static_cast<uint64_t>(a_rows) * a_groups) != DG_OK ||
+        make_map(&map_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<void *>(args.a), K, a_rows,
                  a_groups, static_cast<uint64_t>(K), static_cast<uint64_t>(K) * a_rows, dg::kBlockK,
                  dg::kBlockM, CU_TENSOR_MAP_SWIZZLE_128B) != DG_OK ||
         make_map(&map_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<void *>(args.b), K, N, b_groups,
@@ -823,7 +847,7 @@ int launch(const LaunchArgs &args)
     cfg.stream = static_cast<cudaStream_t>(args.stream);
     cfg.attrs = nullptr;
     cfg.numAttrs = 0;
-    void *kargs[] = {&map_a, &map_b, &p};
+    void *kargs[] = {&map_a, &map_b, &map_d, &p};
     cudaError_t e = cudaLaunchKernelExC(&cfg, fn, kargs);
     if (e != cudaSuccess) {
         cudaGetLastError();

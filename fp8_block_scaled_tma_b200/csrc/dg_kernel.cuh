@@ -18,8 +18,9 @@
 //   warps 4..11     promotion: each thread owns one output row (its TMEM lane) and BN/2
 //                   columns; per K block it loads the fresh partial from TMEM, frees the
 //                   buffer, and adds partial * sa[row] * sb[block] into fp32 registers (sa and
-//                   sb are read with plain loads two K blocks ahead).  After
-//                   the last K block it rounds to bf16 and stores its row segment.
+//                   sb are read with plain loads two K blocks ahead).  After the last K
+//                   block it rounds to bf16 and hands its 32 rows to TMA stores through a
+//                   small staging ring in shared memory.
 // Every wait is bounded by a %globaltimer limit; on expiry the kernel records DG_ERR_TIMEOUT,
 // drains its outstanding copies and MMAs, frees tensor memory and returns.
 #pragma once
@@ -314,10 +315,100 @@ __device__ __forceinline__ bool promote_tile(float (&acc)[NCOLS], const float *s
     return true;
 }
 
+// ---- epilogue -------------------------------------------------------------------------------
+// A promotion warp owns 32 output rows x kCols columns of a tile.  It rounds them to bf16 into a
+// ring of kEpiBufs staging boxes in shared memory (32 rows x 16 columns each) and hands every
+// box to the TMA engine as an asynchronous store, so the warp goes back to promoting the next
+// tile while the copy engine writes whole 32-byte sectors of D.  (Direct per-row stores from
+// the promotion threads touch 32 rows per instruction and cost more time than the promotion of
+// a short-K tile.)  A box row is 32 bytes; with the 32-byte swizzle the 16-byte chunk index is
+// XORed with address bit 7 (bit 2 of the row), which puts the warp's 16-byte shared stores on
+// distinct banks.  Row-masked warps (a partial masked or contiguous tile) store directly.
+constexpr int kEpiCols = 16;
+constexpr int kEpiRows = 32;
+constexpr int kEpiBoxBytes = kEpiRows * kEpiCols * 2;                    // 1 KB
+constexpr int kEpiBufs = 3;
+constexpr int kEpiWarpBytes = kEpiBufs * kEpiBoxBytes;
+constexpr int kEpiBytes = kNumMathWarps * kEpiWarpBytes;                 // 24 KB per CTA
+
+// Stores this warp's rows [y0, y0 + 32) x columns [x0, x0 + NCOLS) of D (a 2-D view of
+// bf16 rows, N wide) through the warp's staging ring `ring`; `ebuf` is the ring position,
+// carried across tiles.  The TMA store clips at the view's bounds.
+template <int NCOLS>
+__device__ __forceinline__ void store_rows_tma(const float (&acc)[NCOLS], const CUtensorMap *tmap_d,
+                                               uint32_t ring, int &ebuf, int x0, int y0, int N,
+                                               int lane)
+{
+    static_assert(NCOLS % kEpiCols == 0, "columns per thread must be a multiple of 16");
+    const uint32_t sw = static_cast<uint32_t>((lane >> 2) & 1);
+#pragma unroll
+    for (int c = 0; c < NCOLS / kEpiCols; ++c) {
+        if (x0 + c * kEpiCols < N) {
+            const uint32_t box = ring + static_cast<uint32_t>(ebuf * kEpiBoxBytes);
+            // the store that last read this box must be done reading it
+            if (lane == 0)
+                ptx::bulk_wait_group_read<kEpiBufs - 1>();
+            __syncwarp();
+            const uint32_t r = box + static_cast<uint32_t>(lane * kEpiCols * 2);
+            const float *v = acc + c * kEpiCols;
+            ptx::st_shared_v4(r + (sw << 4), ptx::pack_bf16x2(v[0], v[1]), ptx::pack_bf16x2(v[2], v[3]),
+                              ptx::pack_bf16x2(v[4], v[5]), ptx::pack_bf16x2(v[6], v[7]));
+            ptx::st_shared_v4(r + ((sw ^ 1u) << 4), ptx::pack_bf16x2(v[8], v[9]),
+                              ptx::pack_bf16x2(v[10], v[11]), ptx::pack_bf16x2(v[12], v[13]),
+                              ptx::pack_bf16x2(v[14], v[15]));
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                ptx::tma_store_2d(tmap_d, box, x0 + c * kEpiCols, y0);
+                ptx::bulk_commit_group();
+            }
+            ebuf = ebuf + 1 == kEpiBufs ? 0 : ebuf + 1;
+        }
+    }
+}
+
+// Direct stores of one thread's row segment (columns [col0, col0 + NCOLS) of row `drow`).
+template <int NCOLS>
+__device__ __forceinline__ void store_row_direct(const float (&acc)[NCOLS], __nv_bfloat16 *drow,
+                                                 int col0, int N)
+{
+#pragma unroll
+    for (int j = 0; j < NCOLS / 8; ++j) {
+        const int col = col0 + 8 * j;
+        if (col < N) {
+            ptx::st_global_v4(drow + col, ptx::pack_bf16x2(acc[8 * j], acc[8 * j + 1]),
+                              ptx::pack_bf16x2(acc[8 * j + 2], acc[8 * j + 3]),
+                              ptx::pack_bf16x2(acc[8 * j + 4], acc[8 * j + 5]),
+                              ptx::pack_bf16x2(acc[8 * j + 6], acc[8 * j + 7]));
+        }
+    }
+}
+
+// Output of one tile by one promotion warp.  `valid` says whether this lane's row may be
+// written and `out_row` is its row in the 2-D view of D.  The TMA path needs all 32 rows
+// writable, except in the dense layout where the store clips rows >= M by itself.
+template <int L, int NCOLS>
+__device__ __forceinline__ void store_tile_rows(const float (&acc)[NCOLS], const Params &p,
+                                                const CUtensorMap *tmap_d, uint32_t ring,
+                                                int &ebuf, bool valid, size_t out_row, int col0,
+                                                int lane)
+{
+    if (!__any_sync(0xffffffffu, valid))
+        return;
+    const bool whole = (L == kDense) || __all_sync(0xffffffffu, valid);
+    if (whole) {
+        const int y0 = __shfl_sync(0xffffffffu, static_cast<int>(out_row), 0);
+        store_rows_tma<NCOLS>(acc, tmap_d, ring, ebuf, col0, y0, p.N, lane);
+    } else if (valid) {
+        store_row_direct<NCOLS>(acc, p.d + out_row * p.N, col0, p.N);
+    }
+}
+
 template <int L, int BN>
 __global__ void __launch_bounds__(kNumThreads, 1)
     dg_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                   const __grid_constant__ CUtensorMap tmap_b, const Params p)
+                   const __grid_constant__ CUtensorMap tmap_b,
+                   const __grid_constant__ CUtensorMap tmap_d, const Params p)
 {
     using C = Cfg<BN>;
     __shared__ SmemCtl ctl;
@@ -354,6 +445,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tmap_a);
         ptx::prefetch_tmap(&tmap_b);
+        ptx::prefetch_tmap(&tmap_d);
     }
     if (warp == 1) {
         ptx::tmem_alloc(ptx::smem_addr(&ctl.tmem_base), kTmemCols);
@@ -495,6 +587,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                                    static_cast<uint32_t>(half * C::kCols);
         constexpr int P1 = C::kPart1;             // columns loaded before the first wait
         constexpr int P2 = C::kCols - P1;         // columns loaded after it (0 if all at once)
+        // this warp's ring of output staging boxes, after the operand stages
+        const uint32_t epi_ring = smem_base + static_cast<uint32_t>(p.stages * C::kStageBytes) +
+                                  static_cast<uint32_t>(mw * kEpiWarpBytes);
+        int ebuf = 0;
         int buf = 0;
         uint32_t bph = 0;
         bool ok = true;
@@ -532,7 +628,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             if (!ok)
                 break;
 
-            // ---- epilogue: bf16 rounding and row-predicated stores ----
+            // ---- epilogue: bf16 rounding, TMA stores of whole warps, direct stores otherwise ----
             const int grow = ti.m0 + row;  // row within the group
             bool valid;
             size_t out_row;
@@ -554,20 +650,12 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 valid = grow < mm;
                 out_row = static_cast<size_t>(ti.g) * p.M + grow;
             }
-            if (valid) {
-                __nv_bfloat16 *drow = p.d + out_row * p.N;
-#pragma unroll
-                for (int j = 0; j < C::kCols / 8; ++j) {
-                    const int col = col0 + 8 * j;
-                    if (col < p.N) {
-                        ptx::st_global_v4(drow + col, ptx::pack_bf16x2(acc[8 * j], acc[8 * j + 1]),
-                                          ptx::pack_bf16x2(acc[8 * j + 2], acc[8 * j + 3]),
-                                          ptx::pack_bf16x2(acc[8 * j + 4], acc[8 * j + 5]),
-                                          ptx::pack_bf16x2(acc[8 * j + 6], acc[8 * j + 7]));
-                    }
-                }
-            }
+            store_tile_rows<L, C::kCols>(acc, p, &tmap_d, epi_ring, ebuf, valid, out_row, col0, lane);
         }
+        // every staged output box is written (and its shared memory read) before exit
+        if (lane == 0)
+            ptx::bulk_wait_group_all();
+        __syncwarp();
     }
 
     // ---- tear-down: everyone is past its last tcgen05 operation ----------------------------

@@ -13,7 +13,8 @@
 //     each 128-wide K block lands in both CTAs' tensor memory, and commits are multicast to both
 //     CTAs' barriers;
 //   - each CTA's promotion warps scale and accumulate their own rows exactly as in the 1-CTA
-//     kernel, and release the TMEM buffer to the even CTA's MMA warp with a cluster arrive.
+//     kernel, release the TMEM buffer to the even CTA's MMA warp with a cluster arrive, and
+//     write the tile through the same TMA-store epilogue.
 // Barriers that collect work of both CTAs (stage full, TMEM buffer empty) live in the even CTA.
 #pragma once
 
@@ -114,7 +115,8 @@ template <int L, int BN>
 __global__ void __launch_bounds__(kNumThreads, 1)
     dg_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         const __grid_constant__ CUtensorMap tmap_b,
-                        const __grid_constant__ CUtensorMap tmap_sfa, const Params p)
+                        const __grid_constant__ CUtensorMap tmap_sfa,
+                        const __grid_constant__ CUtensorMap tmap_d, const Params p)
 {
     using C = PairCfg<BN>;
     constexpr int KS = kKbPerStage;
@@ -166,6 +168,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         ptx::prefetch_tmap(&tmap_a);
         ptx::prefetch_tmap(&tmap_b);
         ptx::prefetch_tmap(&tmap_sfa);
+        ptx::prefetch_tmap(&tmap_d);
     }
     if (warp == 1) {
         ptx::tmem_alloc_pair(ptx::smem_addr(&ctl.tmem_base), kTmemCols);
@@ -341,6 +344,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const uint32_t tempty0 = ptx::map_to_rank(bar_tempty, 0);  // even CTA's buffer barriers
         constexpr int P1 = C::kPart1;
         constexpr int P2 = C::kCols - P1;
+        // this warp's ring of output staging boxes, after the operand stages and the A-scale ring
+        const uint32_t epi_ring = smem_base + static_cast<uint32_t>(sfa_off + kSfaSlots * C::kSfaSlotBytes) +
+                                  static_cast<uint32_t>(mw * kEpiWarpBytes);
+        int ebuf = 0;
         int sj = 0;
         uint32_t sjph = 0;
         int buf = 0;
@@ -431,21 +438,12 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 valid = grow < p.M;
                 out_row = static_cast<size_t>(grow);
             }
-            if (valid) {
-                __nv_bfloat16 *drow = p.d + out_row * p.N;
-#pragma unroll
-                for (int c8 = 0; c8 < C::kCols / 8; ++c8) {
-                    const int col = col0 + 8 * c8;
-                    if (col < p.N) {
-                        ptx::st_global_v4(drow + col,
-                                          ptx::pack_bf16x2(acc[8 * c8], acc[8 * c8 + 1]),
-                                          ptx::pack_bf16x2(acc[8 * c8 + 2], acc[8 * c8 + 3]),
-                                          ptx::pack_bf16x2(acc[8 * c8 + 4], acc[8 * c8 + 5]),
-                                          ptx::pack_bf16x2(acc[8 * c8 + 6], acc[8 * c8 + 7]));
-                    }
-                }
-            }
+            store_tile_rows<L, C::kCols>(acc, p, &tmap_d, epi_ring, ebuf, valid, out_row, col0, lane);
         }
+        // every staged output box is written (and its shared memory read) before exit
+        if (lane == 0)
+            ptx::bulk_wait_group_all();
+        __syncwarp();
     }
 
     // ---- tear-down: both CTAs past their last tcgen05 operation and cross-CTA arrival ----
