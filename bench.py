@@ -43,6 +43,8 @@ METRIC = "FP8 TFLOPS and GB/s per shape at 1 B200; fraction of FP8-peak/HBM roof
 UNIT = "TFLOPS"
 L2_FLUSH_BYTES = 256 << 20
 FP8_PER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor ratio on B200 (4.5 / 2.25 PFLOP/s)
+SPEC_FP8_TFLOPS = 4500.0  # B200 dense FP8 tensor peak (data sheet)
+SPEC_HBM_GBS = 8000.0     # B200 HBM3e bandwidth (data sheet)
 
 
 # ---- workload description ---------------------------------------------------------------------
@@ -120,13 +122,78 @@ def load_peaks():
 
 
 def roofline(g: Gemm, seconds: float, peaks) -> dict:
+    """Per-shape figures: `frac` against the measured denominators (2 x the measured bf16 GEMM
+    for FP8, the measured copy bandwidth for HBM), `frac_spec` against the data-sheet ones."""
     fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16 * 1e12
     bw = peaks["hbm_gbs"] * 1e9
     t_flop, t_mem = g.flops / fp8_peak, g.bytes / bw
+    t_spec = max(g.flops / (SPEC_FP8_TFLOPS * 1e12), g.bytes / (SPEC_HBM_GBS * 1e9))
     bound = "tensor" if t_flop >= t_mem else "hbm"
     return dict(name=g.name, **g.shape, us=seconds * 1e6, tflops=g.flops / seconds / 1e12,
                 gbs=g.bytes / seconds / 1e9, bound=bound, roof_us=max(t_flop, t_mem) * 1e6,
-                frac=max(t_flop, t_mem) / seconds)
+                frac=max(t_flop, t_mem) / seconds, frac_spec=t_spec / seconds)
+
+
+def measure_cublas_fp8(n: int = 8192, reps: int = 10):
+    """A measuring stick for the FP8 tensor peak on this GPU: torch._scaled_mm (cuBLASLt) on an
+    n x n x n e4m3 GEMM with per-tensor scales, median of `reps` event-timed runs after
+    warm-up.  Never on the product path.  Returns TFLOP/s, or None where unsupported."""
+    try:
+        g = torch.Generator(device="cuda")
+        g.manual_seed(7)
+        a = torch.randn(n, n, device="cuda", generator=g).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device="cuda", generator=g).to(torch.float8_e4m3fn)
+        one = torch.ones((), device="cuda")
+        f = lambda: torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        for _ in range(3):
+            f()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e-3)
+        return 2.0 * n ** 3 / statistics.median(ts) / 1e12
+    except Exception:  # an older torch or cuBLAS without FP8: report nothing
+        return None
+
+
+def graph_times(dev, flush, reps: int = 20):
+    """Per-launch device time of each GEMM inside a CUDA graph of `reps` (L2 flush, GEMM) pairs,
+    minus a graph of `reps` flushes alone: the launch-latency-free time of a cold-L2 launch."""
+    def timed(graph):
+        graph.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            graph.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e-3)
+        return statistics.median(ts)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    base = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(base, stream=side):
+        for _ in range(reps):
+            flush.fill_(1)
+    t_flush = timed(base)
+    out = []
+    for d in dev:
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=side):
+            for _ in range(reps):
+                flush.fill_(1)
+                d.launch()
+        out.append(max(0.0, (timed(gr) - t_flush) / reps))
+        del gr
+    del base
+    return out
 
 
 # ---- clocks ---------------------------------------------------------------------------------------
@@ -296,6 +363,16 @@ def run_ours(args, rank, world, local_rank):
     value = aggregate_tflops(flops_step, args.steps, world, total_max)
     peaks = load_peaks()
     shapes = [roofline(g, statistics.mean(p), peaks) for g, p in zip(gemms, per)]
+    if not args.no_graph:
+        # launch-latency-bound shapes (memory-bound, a few microseconds): add the in-graph time
+        idx = [i for i, sh in enumerate(shapes) if sh["bound"] == "hbm"]
+        if idx:
+            gt = graph_times([dev[i] for i in idx], flush)
+            for i, t in zip(idx, gt):
+                if t > 0:
+                    shapes[i].update(graph_us=t * 1e6, graph_frac=shapes[i]["roof_us"] * 1e-6 / t)
+        if dg.poll_device_error(stream) != 0:
+            raise RuntimeError("device error during the graph timing")
     dom = max(range(n), key=lambda i: sum(per[i]))
     dsh = shapes[dom]
     if dsh["bound"] == "tensor":
@@ -307,7 +384,11 @@ def run_ours(args, rank, world, local_rank):
         peak = peaks["hbm_gbs"]
         roof = dict(bound="hbm", achieved=dsh["gbs"], peak=peak, unit="GB/s",
                     frac=dsh["gbs"] / peak, peak_source=f"{peaks['source']} HBM copy")
-    roof.update(kernel=dsh["name"], traffic=args.traffic_bytes, traffic_unit="bytes/launch")
+    roof.update(kernel=dsh["name"], traffic=args.traffic_bytes, traffic_unit="bytes/launch",
+                frac_spec=dsh["frac_spec"])
+    if rank == 0 and not args.no_cublas:
+        # context only: what cuBLAS reaches on an FP8 GEMM on this GPU
+        roof["cublas_fp8_tflops_8192"] = measure_cublas_fp8()
 
     out = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps,
                warmup=args.warmup, ms_per_step=total_max / args.steps * 1e3,
@@ -447,6 +528,8 @@ def main():
     ap.add_argument("--splits", type=int, default=0, help="split-K override (tuning)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph timing of memory-bound shapes")
+    ap.add_argument("--no-cublas", action="store_true", help="skip the cuBLAS FP8 measuring stick")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="dram bytes per launch of the dominant kernel from an ncu capture")

@@ -327,9 +327,9 @@ __device__ __forceinline__ bool promote_tile(float (&acc)[NCOLS], const float *s
 constexpr int kEpiCols = 16;
 constexpr int kEpiRows = 32;
 constexpr int kEpiBoxBytes = kEpiRows * kEpiCols * 2;                    // 1 KB
-constexpr int kEpiBufs = 3;
+constexpr int kEpiBufs = 2;
 constexpr int kEpiWarpBytes = kEpiBufs * kEpiBoxBytes;
-constexpr int kEpiBytes = kNumMathWarps * kEpiWarpBytes;                 // 24 KB per CTA
+constexpr int kEpiBytes = kNumMathWarps * kEpiWarpBytes;                 // 16 KB per CTA
 
 // Stores this warp's rows [y0, y0 + 32) x columns [x0, x0 + NCOLS) of D (a 2-D view of
 // bf16 rows, N wide) through the warp's staging ring `ring`; `ebuf` is the ring position,
