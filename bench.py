@@ -313,6 +313,8 @@ def run_ours(args, rank, world, local_rank):
     gemms, desc = build_workload(args.workload, args.shape)
     if args.block_n or args.stages or args.splits:
         dg.set_config_override(args.block_n, args.stages, args.splits)
+    if args.family:
+        dg.set_kernel_family(args.family)
     dev = [DeviceGemm(dg, g) for g in gemms]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
@@ -526,6 +528,8 @@ def main():
     ap.add_argument("--block-n", type=int, default=0, help="tile override (tuning)")
     ap.add_argument("--stages", type=int, default=0, help="pipeline-stage override (tuning)")
     ap.add_argument("--splits", type=int, default=0, help="split-K override (tuning)")
+    ap.add_argument("--family", type=int, default=0,
+                    help="kernel family override (tuning): 1 one-CTA, 2 CTA pair, 3 split-K")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph timing of memory-bound shapes")
