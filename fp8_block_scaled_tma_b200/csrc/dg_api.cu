@@ -153,17 +153,21 @@ int make_map(CUtensorMap *map, CUtensorMapDataType dt, void *base, uint64_t d0, 
     return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
 }
 
-// 2-D view [rows][N] of the bf16 output for the TMA-store epilogue: one box is 32 rows x 16
-// columns (32-byte rows, 32-byte swizzle), matching the kernels' staging boxes.
-int make_map_d(CUtensorMap *map, void *base, uint64_t N, uint64_t rows)
+// 2-D view [rows][N] of the bf16 output for the TMA-store epilogues: one box is 32 rows x
+// `box_cols` columns (16, 32 or 64), swizzled with the box's row width (32, 64 or 128 bytes) as
+// the kernels' staging boxes are.
+int make_map_d(CUtensorMap *map, void *base, uint64_t N, uint64_t rows, int box_cols = dg::kEpiCols)
 {
     cuuint64_t dims[2] = {N, rows};
     cuuint64_t strides[1] = {N * 2};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(dg::kEpiCols), static_cast<cuuint32_t>(dg::kEpiRows)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(dg::kEpiRows)};
     cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapSwizzle swz = box_cols == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
+                                   : box_cols == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                    : CU_TENSOR_MAP_SWIZZLE_32B;
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
-                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
 }
 
@@ -766,13 +770,15 @@ int launch(const LaunchArgs &args)
             ks.static_bytes = static_cast<int>(fa.sharedSizeBytes);
         }
         const int dyn_cap = info->smem_optin - ks.static_bytes;  // dynamic bytes allowed
-        stages = std::min(dg::kMaxStages, (dyn_cap - 1024 - dg::kEpiBytes) / sbytes);
+        const int epi = dg::whole_tile_epi_bytes(bn);
+        stages = std::min(dg::kMaxStages, (dyn_cap - 1024 - epi) / sbytes);
         if (stages_override > 0)
             stages = std::min(stages, stages_override);
         if (stages < 2)
             return DG_ERR_UNSUPPORTED;
-        // operand stages, the output staging boxes, and slack to align the stages to 1024 bytes
-        dyn_smem = stages * sbytes + dg::kEpiBytes + 1024;
+        // operand stages, the output staging of a whole tile, and slack to align the stages to
+        // 1024 bytes
+        dyn_smem = stages * sbytes + epi + 1024;
         dyn_smem = std::min(std::max(dyn_smem, kMinDynSmem), dyn_cap);
         if (ks.limit_set < dyn_smem) {
             cudaError_t e =
@@ -793,8 +799,11 @@ int launch(const LaunchArgs &args)
     const int a_groups = (args.layout == dg::kMasked) ? G : 1;
     const int b_groups = (args.layout == dg::kDense) ? 1 : G;
     const int m4 = align4(M);
-    CUtensorMap map_a, map_b, map_d;
-    if (make_map_d(&map_d, args.d, N, static_cast<uint64_t>(a_rows) * a_groups) != DG_OK ||
+    CUtensorMap map_a, map_b, map_d64, map_d32, map_d16;
+    const uint64_t d_rows = static_cast<uint64_t>(a_rows) * a_groups;
+    if (make_map_d(&map_d64, args.d, N, d_rows, 64) != DG_OK ||
+        make_map_d(&map_d32, args.d, N, d_rows, 32) != DG_OK ||
+        make_map_d(&map_d16, args.d, N, d_rows, 16) != DG_OK ||
         make_map(&map_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<void *>(args.a), K, a_rows,
                  a_groups, static_cast<uint64_t>(K), static_cast<uint64_t>(K) * a_rows, dg::kBlockK,
                  dg::kBlockM, CU_TENSOR_MAP_SWIZZLE_128B) != DG_OK ||
@@ -847,7 +856,7 @@ int launch(const LaunchArgs &args)
     cfg.stream = static_cast<cudaStream_t>(args.stream);
     cfg.attrs = nullptr;
     cfg.numAttrs = 0;
-    void *kargs[] = {&map_a, &map_b, &map_d, &p};
+    void *kargs[] = {&map_a, &map_b, &map_d64, &map_d32, &map_d16, &p};
     cudaError_t e = cudaLaunchKernelExC(&cfg, fn, kargs);
     if (e != cudaSuccess) {
         cudaGetLastError();

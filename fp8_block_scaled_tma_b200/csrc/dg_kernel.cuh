@@ -19,8 +19,8 @@
 //                   columns; per K block it loads the fresh partial from TMEM, frees the
 //                   buffer, and adds partial * sa[row] * sb[block] into fp32 registers (sa and
 //                   sb are read with plain loads two K blocks ahead).  After the last K
-//                   block it rounds to bf16 and hands its 32 rows to TMA stores through a
-//                   small staging ring in shared memory.
+//                   block it rounds to bf16, stages its 32-row slice of the tile in shared
+//                   memory and writes it with one to three TMA stores.
 // Every wait is bounded by a %globaltimer limit; on expiry the kernel records DG_ERR_TIMEOUT,
 // drains its outstanding copies and MMAs, frees tensor memory and returns.
 #pragma once
@@ -367,6 +367,85 @@ __device__ __forceinline__ void store_rows_tma(const float (&acc)[NCOLS], const 
     }
 }
 
+// ---- whole-tile staging (one-CTA kernel) ----
+// Each TMA store costs its issuing thread ~190 cycles and each staging round a proxy fence, so
+// the one-CTA kernel, whose shared memory allows it, stages a warp's whole 32-row slice of the
+// tile at once and writes it with at most three stores: the NCOLS columns split into pieces of
+// 64, 32 and 16 columns (box rows of 128, 64 and 32 bytes, each with the swizzle of its row
+// width, so the warp's 16-byte shared stores hit distinct banks).  The pieces of all warps are
+// grouped by width (all 64-column pieces first), which keeps every piece aligned to its swizzle
+// pattern.  The store reading a warp's slice has a whole tile to finish before the warp
+// stages its next slice.
+template <int NCOLS>
+struct EpiPieces {
+    static_assert(NCOLS % 16 == 0, "columns per thread must be a multiple of 16");
+    static constexpr int kN64 = NCOLS / 64;
+    static constexpr int kN32 = (NCOLS % 64) / 32;
+    static constexpr int kN16 = (NCOLS % 32) / 16;
+    static constexpr int kWarp64 = kN64 * kEpiRows * 64 * 2;  // bytes per warp, 64-column pieces
+    static constexpr int kWarp32 = kN32 * kEpiRows * 32 * 2;
+    static constexpr int kWarp16 = kN16 * kEpiRows * 16 * 2;
+    static constexpr int kCtaBytes = kNumMathWarps * (kWarp64 + kWarp32 + kWarp16);
+};
+
+// Host-side twin of EpiPieces<BN / 2>::kCtaBytes.
+constexpr int whole_tile_epi_bytes(int bn)
+{
+    return kNumMathWarps * kEpiRows * (bn / 2) * 2;
+}
+
+// One thread's row (`lane` of the box) of a W-column piece at shared address `piece`, from
+// v[0 .. W).  The 16-byte chunk j of row r lands at chunk j XOR (the row's swizzle phase).
+template <int W>
+__device__ __forceinline__ void stage_piece_row(const float *v, uint32_t piece, int lane)
+{
+    constexpr int kRowBytes = W * 2;
+    const uint32_t row = piece + static_cast<uint32_t>(lane * kRowBytes);
+    const uint32_t sw = static_cast<uint32_t>((lane * kRowBytes) >> 7) & (kRowBytes / 16 - 1);
+#pragma unroll
+    for (int j = 0; j < W / 8; ++j)
+        ptx::st_shared_v4(row + ((static_cast<uint32_t>(j) ^ sw) << 4),
+                          ptx::pack_bf16x2(v[8 * j], v[8 * j + 1]), ptx::pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                          ptx::pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), ptx::pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+}
+
+// Stores this warp's rows [y0, y0 + 32) x columns [x0, x0 + NCOLS) of D through the warp's
+// whole-tile staging: `s64`, `s32`, `s16` are the warp's first piece of each width.
+template <int NCOLS>
+__device__ __forceinline__ void store_rows_whole(const float (&acc)[NCOLS], const CUtensorMap *map64,
+                                                 const CUtensorMap *map32, const CUtensorMap *map16,
+                                                 uint32_t s64, uint32_t s32, uint32_t s16, int x0,
+                                                 int y0, int N, int lane)
+{
+    using E = EpiPieces<NCOLS>;
+    // the stores of this warp's previous tile must be done reading the staging
+    if (lane == 0)
+        ptx::bulk_wait_group_read<0>();
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < E::kN64; ++i)
+        stage_piece_row<64>(acc + 64 * i, s64 + static_cast<uint32_t>(i * kEpiRows * 128), lane);
+    if constexpr (E::kN32 > 0)
+        stage_piece_row<32>(acc + 64 * E::kN64, s32, lane);
+    if constexpr (E::kN16 > 0)
+        stage_piece_row<16>(acc + 64 * E::kN64 + 32 * E::kN32, s16, lane);
+    ptx::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < E::kN64; ++i)
+            if (x0 + 64 * i < N)
+                ptx::tma_store_2d(map64, s64 + static_cast<uint32_t>(i * kEpiRows * 128), x0 + 64 * i, y0);
+        if constexpr (E::kN32 > 0)
+            if (x0 + 64 * E::kN64 < N)
+                ptx::tma_store_2d(map32, s32, x0 + 64 * E::kN64, y0);
+        if constexpr (E::kN16 > 0)
+            if (x0 + 64 * E::kN64 + 32 * E::kN32 < N)
+                ptx::tma_store_2d(map16, s16, x0 + 64 * E::kN64 + 32 * E::kN32, y0);
+        ptx::bulk_commit_group();
+    }
+}
+
 // Direct stores of one thread's row segment (columns [col0, col0 + NCOLS) of row `drow`).
 template <int NCOLS>
 __device__ __forceinline__ void store_row_direct(const float (&acc)[NCOLS], __nv_bfloat16 *drow,
@@ -404,11 +483,32 @@ __device__ __forceinline__ void store_tile_rows(const float (&acc)[NCOLS], const
     }
 }
 
+// store_tile_rows with the whole-tile staging of the one-CTA kernel.
+template <int L, int NCOLS>
+__device__ __forceinline__ void store_tile_rows_whole(const float (&acc)[NCOLS], const Params &p,
+                                                      const CUtensorMap *map64, const CUtensorMap *map32,
+                                                      const CUtensorMap *map16, uint32_t s64,
+                                                      uint32_t s32, uint32_t s16, bool valid,
+                                                      size_t out_row, int col0, int lane)
+{
+    if (!__any_sync(0xffffffffu, valid))
+        return;
+    const bool whole = (L == kDense) || __all_sync(0xffffffffu, valid);
+    if (whole) {
+        const int y0 = __shfl_sync(0xffffffffu, static_cast<int>(out_row), 0);
+        store_rows_whole<NCOLS>(acc, map64, map32, map16, s64, s32, s16, col0, y0, p.N, lane);
+    } else if (valid) {
+        store_row_direct<NCOLS>(acc, p.d + out_row * p.N, col0, p.N);
+    }
+}
+
 template <int L, int BN>
 __global__ void __launch_bounds__(kNumThreads, 1)
     dg_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b,
-                   const __grid_constant__ CUtensorMap tmap_d, const Params p)
+                   const __grid_constant__ CUtensorMap tmap_d64,
+                   const __grid_constant__ CUtensorMap tmap_d32,
+                   const __grid_constant__ CUtensorMap tmap_d16, const Params p)
 {
     using C = Cfg<BN>;
     __shared__ SmemCtl ctl;
@@ -445,7 +545,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tmap_a);
         ptx::prefetch_tmap(&tmap_b);
-        ptx::prefetch_tmap(&tmap_d);
+        ptx::prefetch_tmap(&tmap_d64);
+        ptx::prefetch_tmap(&tmap_d32);
+        ptx::prefetch_tmap(&tmap_d16);
     }
     if (warp == 1) {
         ptx::tmem_alloc(ptx::smem_addr(&ctl.tmem_base), kTmemCols);
@@ -587,10 +689,13 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                                    static_cast<uint32_t>(half * C::kCols);
         constexpr int P1 = C::kPart1;             // columns loaded before the first wait
         constexpr int P2 = C::kCols - P1;         // columns loaded after it (0 if all at once)
-        // this warp's ring of output staging boxes, after the operand stages
-        const uint32_t epi_ring = smem_base + static_cast<uint32_t>(p.stages * C::kStageBytes) +
-                                  static_cast<uint32_t>(mw * kEpiWarpBytes);
-        int ebuf = 0;
+        // this warp's output staging pieces (64-, 32- and 16-column), after the operand stages
+        using EP = EpiPieces<C::kCols>;
+        const uint32_t epi0 = smem_base + static_cast<uint32_t>(p.stages * C::kStageBytes);
+        const uint32_t s64 = epi0 + static_cast<uint32_t>(mw * EP::kWarp64);
+        const uint32_t s32 = epi0 + static_cast<uint32_t>(kNumMathWarps * EP::kWarp64 + mw * EP::kWarp32);
+        const uint32_t s16 = epi0 + static_cast<uint32_t>(kNumMathWarps * (EP::kWarp64 + EP::kWarp32) +
+                                                          mw * EP::kWarp16);
         int buf = 0;
         uint32_t bph = 0;
         bool ok = true;
@@ -650,7 +755,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 valid = grow < mm;
                 out_row = static_cast<size_t>(ti.g) * p.M + grow;
             }
-            store_tile_rows<L, C::kCols>(acc, p, &tmap_d, epi_ring, ebuf, valid, out_row, col0, lane);
+            store_tile_rows_whole<L, C::kCols>(acc, p, &tmap_d64, &tmap_d32, &tmap_d16, s64, s32, s16,
+                                               valid, out_row, col0, lane);
         }
         // every staged output box is written (and its shared memory read) before exit
         if (lane == 0)
