@@ -326,7 +326,8 @@ bool choose_splitk(int M, int N, int K, int sms, int bn_fixed, int s_fixed, Capa
     const int m_tiles = (M + dg::kBlockM - 1) / dg::kBlockM;
     double best = 1e300;
     bool found = false;
-    for (int bn = 256; bn >= 64; bn -= 32) {
+    // BN below 128 is searched only when forced: the fitted model below covers 128..256
+    for (int bn = 256; bn >= (bn_fixed != 0 ? 64 : 128); bn -= 32) {
         if (bn_fixed != 0 && bn != bn_fixed)
             continue;
         const long long tiles = static_cast<long long>(m_tiles) * ((N + bn - 1) / bn);
@@ -339,12 +340,17 @@ bool choose_splitk(int M, int N, int K, int sms, int bn_fixed, int s_fixed, Capa
             // every cluster of the grid must be resident at once (one wave)
             if (tiles > capacity(bn, S))
                 continue;
+            // Time model (ns), least-squares fitted to B200 timings of every (BN, S) on ten
+            // memory-bound shapes (M = 64 / 128): a CTA walks its K blocks at ~(537 + 2.85 BN)
+            // cycles each (the TMEM buffer round trip of the two-level accumulation), all CTAs
+            // together cannot beat HBM, and with S > 1 the cluster barriers and the reduction
+            // through distributed shared memory cost ~0.26 us per split plus ~0.14 ns per
+            // partial element of a slice.  (A fixed per-launch cost does not change the choice.)
             const int kb_per = (num_kb + S - 1) / S;
-            const double t_tma = kb_per * (16384.0 + bn * 128.0) / 100.0;                 // ns
+            const double t_kb = kb_per * (537.0 + 2.85 * bn) / 1.9;
             const double t_hbm = (static_cast<double>(N) * K + static_cast<double>(M) * K) / 6500.0;
-            const double t_mma = kb_per * std::max(2.0 * bn, 230.0) / 1.9;
-            const double t_red = S > 1 ? 300.0 + 100.0 * S : 0.0;
-            const double t = std::max(t_tma, std::max(t_hbm, t_mma)) + 1500.0 + t_red;
+            const double t_red = S > 1 ? 263.0 * S + 0.139 * bn * std::min(M, dg::kBlockM) : 0.0;
+            const double t = std::max(t_kb, t_hbm) + t_red;
             if (t < best - 1e-9) {
                 best = t;
                 bn_out = bn;
@@ -719,12 +725,21 @@ int launch(const LaunchArgs &args)
                 n = sms / cs;
             return std::min<long long>(n, sms / cs);
         };
-        if (choose_splitk(M, N, K, sms, bn, splits_override, capacity, sbn, S))
-            return launch_splitk(args, dev, info, sbn, S, stages_override, timeout);
+        if (choose_splitk(M, N, K, sms, bn, splits_override, capacity, sbn, S)) {
+            if (S > 1 || pair_mode == 3)
+                return launch_splitk(args, dev, info, sbn, S, stages_override, timeout);
+            // one split: the one-CTA kernel does the same work without the reduction round
+            // trip through shared memory
+            if (bn == 0)
+                bn = sbn;
+        }
     }
     // CTA pairs (cta_group::2) for the dense and masked layouts: 256-row tiles whose B half is
-    // loaded by each CTA.  Auto mode uses them when a tile of 256 rows is mostly useful and, for
-    // dense problems, K is long (kPairMinKBlocks).
+    // loaded by each CTA.  Auto mode uses them for dense problems with more than 192 rows and
+    // long K (kPairMinKBlocks).  Masked problems stay on the one-CTA kernel: they are bound by
+    // streaming each expert's B once, and a one-CTA tile takes in all BN rows of B per K block
+    // where a pair tile splits them over two SMs (measured on B200, G=32, M_max=256, N=4096,
+    // K=7168: 236 us one-CTA vs 258 us pair, interleaved runs).  Family 2 still forces pairs.
     bool use_pair = false;
     if (args.layout != dg::kContiguous && sms >= 2 && pair_mode != 1 && pair_mode != 3) {
         if (pair_mode == 2)
@@ -732,7 +747,7 @@ int launch(const LaunchArgs &args)
         else if (args.layout == dg::kDense)
             use_pair = M > 192 && num_kb >= kPairMinKBlocks;
         else
-            use_pair = args.expected_m == 0 || args.expected_m > 64;
+            use_pair = false;  // masked: the one-CTA kernel measured ahead (see below)
         if (bn != 0 && pick_pair_kernel(args.layout, bn) == nullptr)
             use_pair = false;  // the block_n override names a tile the pair kernel lacks
     }

@@ -44,13 +44,15 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, float a, float b, fl
                  : "memory");
 }
 
+// Load from a peer's shared memory.  No "memory" clobber, so that a thread can keep many of
+// these in flight and sum later; volatile keeps them after the cluster barrier (also volatile)
+// that publishes the peers' partials.
 __device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t cluster_addr)
 {
     float4 v;
     asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
                  : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(cluster_addr)
-                 : "memory");
+                 : "r"(cluster_addr));
     return v;
 }
 
@@ -108,6 +110,28 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         ptx::prefetch_tmap(&tmap_a);
         ptx::prefetch_tmap(&tmap_b);
     }
+    // The producer issues its first stages at once: they need only this CTA's barriers, which
+    // its own lane 0 has just initialised, so the DRAM latency of the first loads overlaps the
+    // TMEM allocation and the block barrier.  The stage ring then continues from there.
+    uint32_t n_op = 0;  // producer: operand loads issued
+    int ps = 0;         // producer: next stage
+    uint32_t pph = 0;   // producer: its phase
+    if (warp == 0) {
+        __syncwarp();
+        const int pre = min(p.stages, (nkb + KS - 1) / KS);
+        if (ptx::elect_one()) {
+            for (int i = 0; i < pre; ++i) {
+                const uint32_t fb = bar_full + 8 * i;
+                ptx::mbar_arrive_expect_tx(fb, C::kTxBytes);
+                ptx::tma_load_4d(stage_a(i), &tmap_a, fb, 0, m0, kb_begin + i * KS, 0);
+                ptx::tma_load_4d(stage_b(i), &tmap_b, fb, 0, n0, kb_begin + i * KS, 0);
+            }
+        }
+        __syncwarp();
+        n_op = static_cast<uint32_t>(pre);
+        ps = pre == p.stages ? 0 : pre;
+        pph = pre == p.stages ? 1u : 0u;
+    }
     if (warp == 1) {
         ptx::tmem_alloc(ptx::smem_addr(&ctl.tmem_base), kTmemCols);
         ptx::tmem_relinquish();
@@ -123,11 +147,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     if (warp < kFirstMathWarp) {
         ptx::setmaxnreg_dec<40>();
         if (warp == 0) {
-            // ---------------- TMA producer ----------------
-            uint32_t n_op = 0;
-            int s = 0;
-            uint32_t ph = 0;
-            for (int kb0 = kb_begin; kb0 < kb_end; kb0 += KS) {
+            // ---------------- TMA producer (after the stages issued during set-up) ----------------
+            int s = ps;
+            uint32_t ph = pph;
+            for (int kb0 = kb_begin + static_cast<int>(n_op) * KS; kb0 < kb_end; kb0 += KS) {
                 if (!__all_sync(0xffffffffu, wait_one(bar_empty + 8 * s, ph ^ 1, p, abort_flag)))
                     break;
                 if (ptx::elect_one()) {
@@ -257,28 +280,52 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         ptx::cluster_sync();  // every CTA's partial is in place
 
         // ---- reduction of row slice r over the S partials, fixed order ----
+        // Each thread loads the S partials of kBatch 4-column chunks before summing any, so
+        // that up to kBatch * S remote loads are in flight (one at a time is latency-bound).
         const int rows_per = (rows_valid + S - 1) / S;
         const int r_begin = r * rows_per;
         const int r_end = min(rows_valid, r_begin + rows_per);
-        const int chunks_per_row = BN / 4;
-        const int n_chunks = (r_end > r_begin ? r_end - r_begin : 0) * chunks_per_row;
+        constexpr int kChunksPerRow = BN / 4;
+        constexpr int kThreads = kNumMathWarps * 32;
+        constexpr int kBatch = 4;
+        const int n_chunks = (r_end > r_begin ? r_end - r_begin : 0) * kChunksPerRow;
         const int t = threadIdx.x - kFirstMathWarp * 32;  // 0 .. 255
-        for (int ci = t; ci < n_chunks; ci += kNumMathWarps * 32) {
-            const int rr = r_begin + ci / chunks_per_row;
-            const int cc = (ci % chunks_per_row) * 4;
-            const int col = n0 + cc;
-            const uint32_t local = smem_base + static_cast<uint32_t>((rr * C::kPartLd + cc) * 4);
-            float4 sum = ld_shared_cluster_v4(ptx::map_to_rank(local, 0));
-            for (int s2 = 1; s2 < S; ++s2) {
-                const float4 v = ld_shared_cluster_v4(ptx::map_to_rank(local, static_cast<uint32_t>(s2)));
-                sum.x += v.x;
-                sum.y += v.y;
-                sum.z += v.z;
-                sum.w += v.w;
+        for (int c0 = t; c0 < n_chunks; c0 += kBatch * kThreads) {
+            float4 v[kBatch][kMaxSplits];
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) {
+                const int ci = c0 + j * kThreads;
+                if (ci < n_chunks) {
+                    const int rr = r_begin + ci / kChunksPerRow;
+                    const int cc = (ci % kChunksPerRow) * 4;
+                    const uint32_t local = smem_base + static_cast<uint32_t>((rr * C::kPartLd + cc) * 4);
+#pragma unroll
+                    for (int s2 = 0; s2 < kMaxSplits; ++s2)
+                        if (s2 < S)
+                            v[j][s2] = ld_shared_cluster_v4(ptx::map_to_rank(local, static_cast<uint32_t>(s2)));
+                }
             }
-            if (col < p.N) {
-                __nv_bfloat16 *dst = p.d + static_cast<size_t>(m0 + rr) * p.N + col;
-                st_global_v2(dst, ptx::pack_bf16x2(sum.x, sum.y), ptx::pack_bf16x2(sum.z, sum.w));
+#pragma unroll
+            for (int j = 0; j < kBatch; ++j) {
+                const int ci = c0 + j * kThreads;
+                if (ci < n_chunks) {
+                    const int rr = r_begin + ci / kChunksPerRow;
+                    const int col = n0 + (ci % kChunksPerRow) * 4;
+                    float4 sum = v[j][0];
+#pragma unroll
+                    for (int s2 = 1; s2 < kMaxSplits; ++s2) {
+                        if (s2 < S) {
+                            sum.x += v[j][s2].x;
+                            sum.y += v[j][s2].y;
+                            sum.z += v[j][s2].z;
+                            sum.w += v[j][s2].w;
+                        }
+                    }
+                    if (col < p.N) {
+                        __nv_bfloat16 *dst = p.d + static_cast<size_t>(m0 + rr) * p.N + col;
+                        st_global_v2(dst, ptx::pack_bf16x2(sum.x, sum.y), ptx::pack_bf16x2(sum.z, sum.w));
+                    }
+                }
             }
         }
         ptx::cluster_sync();  // peers are done reading this CTA's partial
