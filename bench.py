@@ -160,6 +160,30 @@ def measure_cublas_fp8(n: int = 8192, reps: int = 10):
         return None
 
 
+def back_to_back(dg, dev, flush, gate_cycles: int, reps: int = 10) -> dict:
+    """The whole step enqueued back to back (no event between GEMMs), L2 flushed before it,
+    timed by one event pair: with programmatic dependent launch off and on.  Each kernel's
+    on-chip set-up can then overlap the previous kernel's tail."""
+    stream = torch.cuda.current_stream()
+    out = dict(gemms=len(dev))
+    for key, on in (("pdl_off_ms", False), ("pdl_on_ms", True)):
+        prev = dg.set_pdl(on)
+        ts = []
+        for r in range(reps + 2):
+            torch.cuda._sleep(gate_cycles)
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for d in dev:
+                d.launch(stream)
+            e1.record(stream)
+            stream.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        dg.set_pdl(prev)
+        out[key] = statistics.mean(ts[2:])
+    return out
+
+
 def graph_times(dev, flush, reps: int = 20):
     """Per-launch device time of each GEMM inside a CUDA graph of `reps` (L2 flush, GEMM) pairs,
     minus a graph of `reps` flushes alone: the launch-latency-free time of a cold-L2 launch."""
@@ -375,6 +399,12 @@ def run_ours(args, rank, world, local_rank):
                     shapes[i].update(graph_us=t * 1e6, graph_frac=shapes[i]["roof_us"] * 1e-6 / t)
         if dg.poll_device_error(stream) != 0:
             raise RuntimeError("device error during the graph timing")
+    if not args.no_graph:
+        b2b = back_to_back(dg, dev, flush, gate[0])
+        if dg.poll_device_error(stream) != 0:
+            raise RuntimeError("device error during the back-to-back timing")
+    else:
+        b2b = None
     dom = max(range(n), key=lambda i: sum(per[i]))
     dsh = shapes[dom]
     if dsh["bound"] == "tensor":
@@ -402,7 +432,7 @@ def run_ours(args, rank, world, local_rank):
                                   "step is enqueued behind a bounded sleep kernel",
                            parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
                gbs=world * bytes_step * args.steps / total_max / 1e9,
-               roofline=roof, per_shape=shapes, gpu_launches=n * args.steps,
+               roofline=roof, per_shape=shapes, back_to_back=b2b, gpu_launches=n * args.steps,
                clocks=clk.summary(), last_launch=launch_info)
 
     # e2e through the public API with host buffers

@@ -73,6 +73,8 @@ def _load() -> ctypes.CDLL:
     lib.dg_set_fault_injection.restype = i
     lib.dg_set_kernel_family.argtypes = [i]
     lib.dg_set_kernel_family.restype = i
+    lib.dg_set_pdl.argtypes = [i]
+    lib.dg_set_pdl.restype = i
     ipp = ctypes.POINTER(ctypes.c_int)
     lib.dg_get_last_launch.argtypes = [ipp, ipp, ipp, ipp, ipp, ipp]
     lib.dg_get_last_launch.restype = i
@@ -187,6 +189,15 @@ def set_kernel_family(family: int) -> int:
     if r < 0:
         raise DGError(r, "dg_set_kernel_family")
     return r
+
+
+def set_pdl(enable: bool) -> bool:
+    """Programmatic dependent launch of the GEMMs (on by default): back-to-back kernels overlap
+    their on-chip set-up with the previous kernel's tail.  Returns the previous setting."""
+    r = lib.dg_set_pdl(1 if enable else 0)
+    if r < 0:
+        raise DGError(r, "dg_set_pdl")
+    return bool(r)
 
 
 def get_last_launch() -> dict:

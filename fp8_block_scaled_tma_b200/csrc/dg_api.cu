@@ -49,6 +49,7 @@ int g_override_bn = 0;
 int g_override_stages = 0;
 int g_override_splits = 0;
 int g_inject_stall = 0;
+int g_pdl = 1;  // launch with programmatic stream serialisation (dg_set_pdl)
 // clusters of each size (index = cluster size, 1..8) that can be resident at once, per device
 // and kernel family; 0 = not queried yet
 int g_max_clusters[kMaxDevices][3][9];
@@ -68,6 +69,23 @@ bool debug_enabled()
         v = (e && e[0] && e[0] != '0') ? 1 : 0;
     }
     return v == 1;
+}
+
+// Appends the programmatic-dependent-launch attribute when it is enabled: the kernel may then
+// be scheduled while the previous kernel of the stream finishes; every kernel waits for it
+// (griddepcontrol.wait) before touching global memory, so stream order is kept.
+int add_pdl_attr(cudaLaunchAttribute *attr, int n)
+{
+    int on;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        on = g_pdl;
+    }
+    if (!on)
+        return n;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    return n + 1;
 }
 
 // Per-device set-up: checks for sm_100, reads SM count and shared-memory limit, and resolves
@@ -503,13 +521,13 @@ int launch_splitk(const LaunchArgs &args, int dev, DeviceInfo *info, int bn, int
     cfg.blockDim = dim3(dg::kNumThreads, 1, 1);
     cfg.dynamicSmemBytes = dyn_smem;
     cfg.stream = static_cast<cudaStream_t>(args.stream);
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = S;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = add_pdl_attr(attr, 1);
     void *kargs[] = {&map_a, &map_b, &p};
     cudaError_t e = cudaLaunchKernelExC(&cfg, fn, kargs);
     if (e != cudaSuccess) {
@@ -646,13 +664,13 @@ int launch_pair(const LaunchArgs &args, int dev, DeviceInfo *info, int sms, int 
     cfg.blockDim = dim3(dg::kNumThreads, 1, 1);
     cfg.dynamicSmemBytes = dyn_smem;
     cfg.stream = static_cast<cudaStream_t>(args.stream);
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = add_pdl_attr(attr, 1);
     void *kargs[] = {&map_a, &map_b, &map_sfa, &map_d, &p};
     cudaError_t e = cudaLaunchKernelExC(&cfg, fn, kargs);
     if (e != cudaSuccess) {
@@ -869,8 +887,9 @@ int launch(const LaunchArgs &args)
     cfg.blockDim = dim3(dg::kNumThreads, 1, 1);
     cfg.dynamicSmemBytes = dyn_smem;
     cfg.stream = static_cast<cudaStream_t>(args.stream);
-    cfg.attrs = nullptr;
-    cfg.numAttrs = 0;
+    cudaLaunchAttribute attr[1];
+    cfg.attrs = attr;
+    cfg.numAttrs = add_pdl_attr(attr, 0);
     void *kargs[] = {&map_a, &map_b, &map_d64, &map_d32, &map_d16, &p};
     cudaError_t e = cudaLaunchKernelExC(&cfg, fn, kargs);
     if (e != cudaSuccess) {
@@ -1088,6 +1107,16 @@ int dg_set_fault_injection(int mode)
     std::lock_guard<std::mutex> lock(g_mutex);
     int prev = g_inject_stall;
     g_inject_stall = mode;
+    return prev;
+}
+
+int dg_set_pdl(int enable)
+{
+    if (enable != 0 && enable != 1)
+        return DG_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int prev = g_pdl;
+    g_pdl = enable;
     return prev;
 }
 

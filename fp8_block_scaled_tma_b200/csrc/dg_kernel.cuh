@@ -528,6 +528,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const uint32_t bar_tempty = ptx::smem_addr(&ctl.tmem_empty[0]);
     const uint32_t bar_drain = ptx::smem_addr(&ctl.drain);
     volatile int *abort_flag = &ctl.abort_flag;
+    ptx::griddep_launch_dependents();  // the next grid may start its set-up as SMs free up
 
     // ---- set-up ------------------------------------------------------------------------
     if (threadIdx.x == 0) {
@@ -553,6 +554,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         ptx::tmem_alloc(ptx::smem_addr(&ctl.tmem_base), kTmemCols);
         ptx::tmem_relinquish();
     }
+    // no global memory is touched before the grids this one depends on are complete
+    ptx::griddep_wait();
     if (L == kMasked) {
         if (warp == 2 && lane == 0) {
             // prefix over groups of (m-tiles of the group) * n_tiles

@@ -146,6 +146,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const uint32_t bar_sfull = ptx::smem_addr(&ctl.sfa_full[0]);
     const uint32_t bar_sempty = ptx::smem_addr(&ctl.sfa_empty[0]);
     volatile int *abort_flag = &ctl.abort_flag;
+    ptx::griddep_launch_dependents();  // the next grid may start its set-up as SMs free up
 
     // ---- set-up ------------------------------------------------------------------------
     if (threadIdx.x == 0) {
@@ -174,6 +175,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         ptx::tmem_alloc_pair(ptx::smem_addr(&ctl.tmem_base), kTmemCols);
         ptx::tmem_relinquish_pair();
     }
+    // no global memory is touched before the grids this one depends on are complete
+    ptx::griddep_wait();
     if (L == kMasked) {
         if (warp == 2 && lane == 0) {
             int acc = 0;

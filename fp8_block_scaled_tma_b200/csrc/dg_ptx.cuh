@@ -489,6 +489,23 @@ __device__ __forceinline__ void bulk_wait_group_all()
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// ---- programmatic dependent launch -----------------------------------------------------------
+
+// Lets the next grid in the stream (launched with programmatic stream serialisation) be
+// scheduled before this one completes.  Safe at any point: the dependent still waits for this
+// grid's completion in griddep_wait before it touches global memory.
+__device__ __forceinline__ void griddep_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Waits until the grids this one depends on have completed and their memory operations are
+// visible.  Returns at once when the grid was launched without a programmatic dependency.
+__device__ __forceinline__ void griddep_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 template <uint32_t kRegs>
 __device__ __forceinline__ void setmaxnreg_inc()
 {

@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const uint32_t bar_tempty = ptx::smem_addr(&ctl.tmem_empty[0]);
     const uint32_t bar_drain = ptx::smem_addr(&ctl.drain);
     volatile int *abort_flag = &ctl.abort_flag;
+    ptx::griddep_launch_dependents();  // the next grid may start its set-up as SMs free up
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
@@ -110,6 +111,12 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         ptx::prefetch_tmap(&tmap_a);
         ptx::prefetch_tmap(&tmap_b);
     }
+    if (warp == 1) {
+        ptx::tmem_alloc(ptx::smem_addr(&ctl.tmem_base), kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    // no global memory is touched before the grids this one depends on are complete
+    ptx::griddep_wait();
     // The producer issues its first stages at once: they need only this CTA's barriers, which
     // its own lane 0 has just initialised, so the DRAM latency of the first loads overlaps the
     // TMEM allocation and the block barrier.  The stage ring then continues from there.
@@ -131,10 +138,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         n_op = static_cast<uint32_t>(pre);
         ps = pre == p.stages ? 0 : pre;
         pph = pre == p.stages ? 1u : 0u;
-    }
-    if (warp == 1) {
-        ptx::tmem_alloc(ptx::smem_addr(&ctl.tmem_base), kTmemCols);
-        ptx::tmem_relinquish();
     }
     ptx::tc_fence_before();
     __syncthreads();

@@ -144,10 +144,21 @@ int dg_set_config_override(int block_n, int num_stages, int splits);
  * its expert segments are only 128-row aligned); 3 = the split-K cluster kernel for dense calls
  * whose output tiles fit in one wave (the K blocks of a tile are split over up to 8 CTAs that
  * reduce their fp32 partials through distributed shared memory, in a fixed order).  Automatic
- * mode uses split-K for dense M <= 256, pairs for larger dense M and for masked calls.  Results
- * agree within the parity tolerance whichever family runs.  Returns the previous value, or
- * DG_ERR_INVALID_ARG. */
+ * mode uses split-K for dense M <= 256 when more than one split pays (else the one-CTA kernel),
+ * pairs for dense M > 256 with K >= 96 * 128, and the one-CTA kernels otherwise (contiguous and
+ * masked included).  Results agree within the parity tolerance whichever family runs.  Returns
+ * the previous value, or DG_ERR_INVALID_ARG. */
 int dg_set_kernel_family(int family);
+
+/* Programmatic dependent launch (a Hopper/Blackwell launch feature, not on the pages; on by
+ * default).  When enabled, every GEMM is launched with programmatic stream serialisation: its
+ * CTAs may be scheduled, and run their on-chip set-up (barrier initialisation, tensor-memory
+ * allocation, tensor-map prefetch), while the previous kernel of the stream finishes; each kernel
+ * signals its dependents at entry and executes griddepcontrol.wait before its first access to
+ * global memory, so results and stream ordering are the same with the switch on or off.  The
+ * overlap only happens between back-to-back kernels (an event or memcpy in between is a full
+ * dependency).  enable: 0 or 1.  Returns the previous value, or DG_ERR_INVALID_ARG. */
+int dg_set_pdl(int enable);
 
 /* Describes the most recent launch on this host thread: fills any non-NULL pointer with the
  * chosen block_n, pipeline stages, grid size (CTAs), output tile count, kernel family (1, 2 or

@@ -78,6 +78,9 @@ def test_config_override_validation(dg):
     assert dg.lib.dg_set_fault_injection(2) == dg.DG_ERR_INVALID_ARG
     assert dg.lib.dg_set_fault_injection(0) == dg.DG_OK
     assert dg.lib.dg_set_kernel_family(0) == dg.DG_OK
+    assert dg.lib.dg_set_pdl(2) == dg.DG_ERR_INVALID_ARG
+    prev = dg.set_pdl(False)
+    assert dg.set_pdl(prev) is False
 
 
 def test_timeout_setter(dg):
