@@ -48,6 +48,11 @@ def _load():
     u16p = ctypes.POINTER(ctypes.c_uint16)
     f64p = ctypes.POINTER(ctypes.c_double)
     i64 = ctypes.c_int64
+    lib.orc_e4m3_encode.argtypes = [ctypes.c_float]
+    lib.orc_e4m3_encode.restype = ctypes.c_uint8
+    lib.orc_quantize_1x128.argtypes = [ctypes.POINTER(ctypes.c_uint16), ctypes.c_int64, ctypes.c_int64,
+                                       ctypes.POINTER(ctypes.c_uint8), ctypes.POINTER(ctypes.c_float)]
+    lib.orc_quantize_1x128.restype = ctypes.c_int
     lib.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
     lib.orc_e4m3_decode.restype = ctypes.c_double
     lib.orc_bf16_rne.argtypes = [ctypes.c_double]
@@ -79,6 +84,26 @@ def _as(x, dtype) -> np.ndarray:
 def e4m3_decode(code: int) -> float:
     """Value of one OCP E4M3 ("fn") code, from the format's definition."""
     return float(_load().orc_e4m3_decode(int(code) & 0xFF))
+
+
+def e4m3_encode(x: float) -> int:
+    """fp32 -> E4M3 code, round to nearest even, saturating at 448."""
+    return int(_load().orc_e4m3_encode(float(x)))
+
+
+def quantize_1x128(x_bits: np.ndarray):
+    """Per-token FP8 quantisation.  x_bits: uint16 bf16 bits [M][K].  Returns (codes uint8
+    [M][K], scales float32 [M][K/128])."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    M, K = x.shape
+    q = np.empty((M, K), dtype=np.uint8)
+    sa = np.empty((M, K // 128), dtype=np.float32)
+    r = _load().orc_quantize_1x128(x.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16)), M, K,
+                                   q.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
+                                   sa.ctypes.data_as(ctypes.POINTER(ctypes.c_float)))
+    if r != 0:
+        raise ValueError("orc_quantize_1x128: K must be a multiple of 128")
+    return q, sa
 
 
 def bf16_rne(x: float) -> int:

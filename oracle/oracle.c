@@ -89,6 +89,74 @@ uint16_t orc_bf16_rne(double x)
     return sign | (uint16_t)bits;
 }
 
+/* IEEE-754 round-to-nearest-even of a float to E4M3 with saturation to the largest finite
+ * magnitude (448): the conversion of the per-token quantisation below.  Written from the
+ * format's definition: normal codes (1 + m/8) 2^(e-7) for e = 1..15 (e = 15 only m <= 6),
+ * subnormal codes (m/8) 2^-6; the quantum is 2^-9 below 2^-6 and 2^(E-3) in binade E.  NaN in,
+ * NaN code out; -0 keeps its sign. */
+uint8_t orc_e4m3_encode(float v)
+{
+    if (v != v)
+        return 0x7F;
+    const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs((double)v);
+    if (a >= 448.0)
+        return sign | 0x7E;
+    if (a < ldexp(1.0, -6)) {
+        /* subnormal range: multiples of 2^-9; q = 8 is the smallest normal, code 0x08 */
+        const double q = rint(ldexp(a, 9));
+        return sign | (uint8_t)q;
+    }
+    int e;
+    frexp(a, &e);             /* a = f 2^e, f in [0.5, 1): binade E = e - 1 */
+    int E = e - 1;
+    double q = rint(ldexp(a, 3 - E));   /* in [8, 16] */
+    if (q >= 16.0) {
+        q = 8.0;
+        E += 1;
+    }
+    const int code = ((E + 7) << 3) | ((int)q - 8);
+    return sign | (uint8_t)(code > 0x7E ? 0x7E : code);
+}
+
+/* ---- per-token (1 x 128) FP8 quantisation of bf16 activations ------------------------- */
+
+/* The step before the GEMM (DeepGEMM release write-up, "深入了解DeepGEMM": activations carry
+ * one scale per 1 x 128 tile).  For each row m and K block kb, in fp32:
+ *     amax  = max |x| over the tile
+ *     scale = max(amax, 1e-4) / 448
+ *     q[k]  = e4m3_rne(x[k] / scale)      (saturating at 448)
+ * x is bf16 bits [M][K]; q codes [M][K]; sa the logical scales [M][K/128].  The quotient and
+ * the scale are single fp32 operations, rounded to nearest even, as the GPU kernel computes
+ * them, so the integer codes can be compared bit for bit. */
+int orc_quantize_1x128(const uint16_t *x, int64_t M, int64_t K, uint8_t *q, float *sa)
+{
+    if (K % ORC_BLOCK != 0 || M < 0)
+        return -1;
+    const int64_t kbs = K / ORC_BLOCK;
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t kb = 0; kb < kbs; ++kb) {
+            const uint16_t *xt = x + m * K + kb * ORC_BLOCK;
+            float vals[ORC_BLOCK];
+            float amax = 0.0f;
+            for (int i = 0; i < ORC_BLOCK; ++i) {
+                uint32_t w = (uint32_t)xt[i] << 16;  /* bf16 -> fp32 is exact */
+                float f;
+                memcpy(&f, &w, 4);
+                vals[i] = f;
+                const float a = fabsf(f);
+                if (a > amax)
+                    amax = a;
+            }
+            const float scale = (amax > 1e-4f ? amax : 1e-4f) / 448.0f;
+            sa[m * kbs + kb] = scale;
+            for (int i = 0; i < ORC_BLOCK; ++i)
+                q[m * K + kb * ORC_BLOCK + i] = orc_e4m3_encode(vals[i] / scale);
+        }
+    }
+    return 0;
+}
+
 /* ---- one output row ------------------------------------------------------------------ */
 
 typedef struct {
