@@ -73,6 +73,8 @@ def _load() -> ctypes.CDLL:
     lib.dg_set_fault_injection.restype = i
     lib.dg_set_kernel_family.argtypes = [i]
     lib.dg_set_kernel_family.restype = i
+    lib.dg_quantize_fp8_1x128.argtypes = [vp, vp, fp, i, i, vp]
+    lib.dg_quantize_fp8_1x128.restype = i
     lib.dg_set_pdl.argtypes = [i]
     lib.dg_set_pdl.restype = i
     ipp = ctypes.POINTER(ctypes.c_int)
@@ -244,6 +246,28 @@ def dg_gemm_fp8_fp8_bf16_nt(a, sfa, b, sfb, d, workspace=None, stream=None) -> N
     _check(lib.dg_gemm_fp8_fp8_bf16_nt(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K,
                                        _ptr(workspace), ws, _stream(stream)),
            "dg_gemm_fp8_fp8_bf16_nt")
+
+
+def quantize_fp8_1x128(x, q=None, sfa=None, stream=None):
+    """Per-token FP8 quantisation on the GPU: x bf16 [M,K] -> (q uint8 e4m3 codes [M,K],
+    sfa fp32 [K/128, align4(M)] MN-major, the GEMMs' A-scale layout).  Output tensors may be
+    passed in (they are overwritten); otherwise they are allocated here with torch."""
+    if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous() or x.dim() != 2:
+        raise ValueError("x must be a contiguous 2-D bfloat16 CUDA tensor")
+    M, K = x.shape
+    if K % BLOCK != 0:
+        raise ValueError("K must be a multiple of 128")
+    if q is None:
+        q = torch.empty(M, K, dtype=torch.uint8, device=x.device)
+    _fp8(q, "q")
+    if tuple(q.shape) != (M, K):
+        raise ValueError("q must be [M, K]")
+    if sfa is None:
+        sfa = torch.empty(K // BLOCK, get_tma_aligned_size(M, 4), dtype=torch.float32, device=x.device)
+    _f32(sfa, "sfa", (K // BLOCK, get_tma_aligned_size(M, 4)))
+    _check(lib.dg_quantize_fp8_1x128(_ptr(x), _ptr(q), _ptr(sfa), M, K, _stream(stream)),
+           "dg_quantize_fp8_1x128")
+    return q, sfa
 
 
 def dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(a, sfa, b, sfb, d, m_indices, workspace=None,

@@ -13,6 +13,7 @@
 #include "../../include/dg.h"
 #include "dg_kernel.cuh"
 #include "dg_pair_kernel.cuh"
+#include "dg_quant_kernel.cuh"
 #include "dg_splitk_kernel.cuh"
 
 namespace {
@@ -924,9 +925,52 @@ int check_common(const void *a, const float *sfa, const void *b, const float *sf
     return DG_OK;
 }
 
+int launch_quantize(const void *x, void *q, float *sfa, int M, int K, void *stream)
+{
+    int dev = 0;
+    DeviceInfo *info = nullptr;
+    int st = device_setup(dev, info);
+    if (st != DG_OK)
+        return st;
+    const long long blocks_x = (static_cast<long long>(M) + dg::kQuantRowsPerBlock - 1) / dg::kQuantRowsPerBlock;
+    if (blocks_x > 0x7FFFFFFFLL || K / dg::kBlockK > 65535)
+        return DG_ERR_INVALID_ARG;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks_x), static_cast<unsigned>(K / dg::kBlockK), 1);
+    cfg.blockDim = dim3(dg::kQuantThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    cfg.attrs = attr;
+    cfg.numAttrs = add_pdl_attr(attr, 0);
+    const __nv_bfloat16 *xp = static_cast<const __nv_bfloat16 *>(x);
+    uint8_t *qp = static_cast<uint8_t *>(q);
+    int m4 = align4(M);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, dg::dg_quantize_1x128_kernel, xp, qp, sfa, M, K, m4);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        if (debug_enabled())
+            std::fprintf(stderr, "[dg] quantize launch failed: %s\n", cudaGetErrorString(e));
+        return DG_ERR_CUDA;
+    }
+    return DG_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+int dg_quantize_fp8_1x128(const void *x, void *q, float *sfa, int M, int K, void *stream)
+{
+    if (M < 0 || K <= 0 || K % dg::kBlockK != 0)
+        return DG_ERR_INVALID_ARG;
+    if (M == 0)
+        return DG_OK;
+    if (!x || !q || !sfa || !aligned16(x) || !aligned16(q) || !aligned16(sfa))
+        return DG_ERR_INVALID_ARG;
+    return launch_quantize(x, q, sfa, M, K, stream);
+}
 
 int dg_gemm_fp8_fp8_bf16_nt(const void *a, const float *sfa, const void *b, const float *sfb,
                             void *d, int M, int N, int K, void *workspace, size_t workspace_bytes,

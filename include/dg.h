@@ -94,6 +94,22 @@ int dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked(const void *a, const float *sfa, co
                                              void *workspace, size_t workspace_bytes,
                                              void *stream);
 
+/* Per-token FP8 quantisation of activations: the step that produces the GEMMs' A operand and
+ * its scales (the fine-grained 1 x 128 activation scaling of "深入了解DeepGEMM", written in the
+ * TMA-aligned scale layout that the utility functions of "如何使用" serve).  For each row m and
+ * K block kb, in fp32 with IEEE round-to-nearest-even operations:
+ *     amax    = max(max |x[m][128 kb .. 128 kb + 127]|, 1e-4)
+ *     scale   = amax / 448                     (written to sfa)
+ *     q[m][k] = e4m3(x[m][k] * (448 / amax)), round to nearest even, saturating at +-448
+ *   x    bf16 [M][K] row-major (device); finite values (NaN / inf give unspecified codes)
+ *   q    e4m3 codes [M][K] row-major (device, written)
+ *   sfa  fp32 [K/128][align4(M)], MN-major: the layout every GEMM here reads (device, written;
+ *        the padding entries of rows M .. align4(M)-1 are not written)
+ *   M >= 0 (0 launches nothing), K > 0 and K % 128 == 0, pointers 16-byte aligned, K/128 <=
+ *   65535.  The caller owns all buffers; nothing is allocated; asynchronous on `stream`.
+ * Returns DG_OK, DG_ERR_INVALID_ARG (nothing launched), DG_ERR_UNSUPPORTED or DG_ERR_CUDA. */
+int dg_quantize_fp8_1x128(const void *x, void *q, float *sfa, int M, int K, void *stream);
+
 /* The SM-count utility of "如何使用": caps the number of SMs the persistent kernels occupy so
  * that other work (for example communication kernels) can run beside them.  n <= 0 restores
  * "all SMs".  Returns the previous cap (0 = all). */

@@ -123,12 +123,13 @@ uint8_t orc_e4m3_encode(float v)
 
 /* The step before the GEMM (DeepGEMM release write-up, "深入了解DeepGEMM": activations carry
  * one scale per 1 x 128 tile).  For each row m and K block kb, in fp32:
- *     amax  = max |x| over the tile
- *     scale = max(amax, 1e-4) / 448
- *     q[k]  = e4m3_rne(x[k] / scale)      (saturating at 448)
- * x is bf16 bits [M][K]; q codes [M][K]; sa the logical scales [M][K/128].  The quotient and
- * the scale are single fp32 operations, rounded to nearest even, as the GPU kernel computes
- * them, so the integer codes can be compared bit for bit. */
+ *     amax   = max(max |x| over the tile, 1e-4)
+ *     factor = 448 / amax                 (one division per tile)
+ *     scale  = amax / 448                 (the dequantisation scale the GEMM reads)
+ *     q[k]   = e4m3_rne(x[k] * factor)    (saturating at 448)
+ * x is bf16 bits [M][K]; q codes [M][K]; sa the logical scales [M][K/128].  Every step is a
+ * single fp32 operation rounded to nearest even, as the GPU kernel computes it, so the integer
+ * codes and the scales can be compared bit for bit. */
 int orc_quantize_1x128(const uint16_t *x, int64_t M, int64_t K, uint8_t *q, float *sa)
 {
     if (K % ORC_BLOCK != 0 || M < 0)
@@ -148,10 +149,11 @@ int orc_quantize_1x128(const uint16_t *x, int64_t M, int64_t K, uint8_t *q, floa
                 if (a > amax)
                     amax = a;
             }
-            const float scale = (amax > 1e-4f ? amax : 1e-4f) / 448.0f;
-            sa[m * kbs + kb] = scale;
+            const float amax_c = amax > 1e-4f ? amax : 1e-4f;
+            const float factor = 448.0f / amax_c;
+            sa[m * kbs + kb] = amax_c / 448.0f;
             for (int i = 0; i < ORC_BLOCK; ++i)
-                q[m * K + kb * ORC_BLOCK + i] = orc_e4m3_encode(vals[i] / scale);
+                q[m * K + kb * ORC_BLOCK + i] = orc_e4m3_encode(vals[i] * factor);
         }
     }
     return 0;

@@ -152,3 +152,12 @@ def test_sfa_layout_helper(dg):
     mn3 = dg.sfa_mn_major(sa3)
     assert mn3.shape == (2, 2, 8)
     assert torch.equal(mn3[1, :, :5], sa3[1].t())
+
+
+def test_quantize_rejects_bad_arguments(dg):
+    L = dg.lib
+    assert L.dg_quantize_fp8_1x128(FAKE, FAKE, FAKE, 4, 100, None) == dg.DG_ERR_INVALID_ARG   # K % 128
+    assert L.dg_quantize_fp8_1x128(FAKE, FAKE, FAKE, -1, 128, None) == dg.DG_ERR_INVALID_ARG  # M < 0
+    assert L.dg_quantize_fp8_1x128(FAKE + 4, FAKE, FAKE, 4, 128, None) == dg.DG_ERR_INVALID_ARG
+    assert L.dg_quantize_fp8_1x128(None, FAKE, FAKE, 4, 128, None) == dg.DG_ERR_INVALID_ARG
+    assert L.dg_quantize_fp8_1x128(None, None, None, 0, 128, None) == dg.DG_OK  # empty: no-op

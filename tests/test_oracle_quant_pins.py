@@ -3,7 +3,7 @@ per 1 x 128 tile of the activations, DeepGEMM release write-up, "深入了解Dee
 encoder is checked against the format's own grid (every code round-trips, ties go to the even
 code) and against torch's independent float8_e4m3fn cast; the quantiser against properties that
 any correct implementation has (the largest element maps to +-448, all-zero tiles use the 1e-4
-floor, every element is the nearest grid point of x / scale) and against a numpy/torch
+floor, every element is the nearest grid point of x * (448 / amax)) and against a numpy/torch
 composition on random data."""
 from __future__ import annotations
 
@@ -91,13 +91,14 @@ def test_quantise_properties():
         for kb in range(K // 128):
             t = xf[m, kb * 128:(kb + 1) * 128]
             amax = np.float32(np.abs(t).max())
-            s = np.float32(max(amax, np.float32(1e-4))) / np.float32(448.0)
+            amax_c = np.float32(max(amax, np.float32(1e-4)))
+            s = amax_c / np.float32(448.0)
             assert sa[m, kb] == s
             codes = q[m, kb * 128:(kb + 1) * 128]
             if amax >= 1e-4:
                 assert np.any((codes & 0x7F) == 0x7E)  # the largest element maps to +-448
-            # each code is the nearest grid point of x / s (ties to even)
-            quot = (t / s).astype(np.float32)
+            # each code is the nearest grid point of x * (448 / amax) (ties to even)
+            quot = (t * (np.float32(448.0) / amax_c)).astype(np.float32)
             dec = np.array([oracle.e4m3_decode(int(c)) for c in codes])
             for v, d in zip(quot, dec):
                 v = float(v)
@@ -116,9 +117,10 @@ def test_quantise_matches_numpy_torch_composition():
     x[rng.random((M, K)) < 0.01] *= 50.0
     bits = _bf16_bits(x)
     xf = _bits_to_f32(bits).reshape(M, K // 128, 128)
-    amax = np.abs(xf).max(axis=2)
-    s = np.maximum(amax, np.float32(1e-4)).astype(np.float32) / np.float32(448.0)
-    quot = (xf / s[:, :, None]).astype(np.float32).reshape(M, K)
+    amax = np.maximum(np.abs(xf).max(axis=2), np.float32(1e-4)).astype(np.float32)
+    s = amax / np.float32(448.0)
+    factor = np.float32(448.0) / amax
+    quot = (xf * factor[:, :, None]).astype(np.float32).reshape(M, K)
     ref_q = torch.from_numpy(np.clip(quot, -448, 448)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     q, sa = oracle.quantize_1x128(bits)
     assert np.array_equal(sa, s)
