@@ -53,6 +53,10 @@ def _load():
     lib.orc_quantize_1x128.argtypes = [ctypes.POINTER(ctypes.c_uint16), ctypes.c_int64, ctypes.c_int64,
                                        ctypes.POINTER(ctypes.c_uint8), ctypes.POINTER(ctypes.c_float)]
     lib.orc_quantize_1x128.restype = ctypes.c_int
+    lib.orc_swiglu_quantize.argtypes = [ctypes.POINTER(ctypes.c_uint16), ctypes.c_int64, ctypes.c_int64,
+                                        ctypes.POINTER(ctypes.c_uint8), ctypes.POINTER(ctypes.c_uint8),
+                                        ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]
+    lib.orc_swiglu_quantize.restype = ctypes.c_int
     lib.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
     lib.orc_e4m3_decode.restype = ctypes.c_double
     lib.orc_bf16_rne.argtypes = [ctypes.c_double]
@@ -104,6 +108,29 @@ def quantize_1x128(x_bits: np.ndarray):
     if r != 0:
         raise ValueError("orc_quantize_1x128: K must be a multiple of 128")
     return q, sa
+
+
+def swiglu_quantize(h_bits: np.ndarray, row_valid: np.ndarray | None = None):
+    """SwiGLU then per-token FP8 quantisation.  h_bits: uint16 bf16 bits [M][2I] (gate half,
+    then up half).  Returns (codes uint8 [M][I], scales float32 [M][I/128], y float32 [M][I]);
+    rows with row_valid == 0 are left as 0 / 0 / NaN."""
+    h = np.ascontiguousarray(h_bits, dtype=np.uint16)
+    M, two_i = h.shape
+    I = two_i // 2
+    q = np.zeros((M, I), dtype=np.uint8)
+    sa = np.zeros((M, I // 128), dtype=np.float32)
+    y = np.full((M, I), np.nan, dtype=np.float32)
+    rv = None
+    if row_valid is not None:
+        rv = np.ascontiguousarray(row_valid, dtype=np.uint8)
+    r = _load().orc_swiglu_quantize(h.ctypes.data_as(ctypes.POINTER(ctypes.c_uint16)), M, I,
+                                    None if rv is None else rv.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
+                                    q.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
+                                    sa.ctypes.data_as(ctypes.POINTER(ctypes.c_float)),
+                                    y.ctypes.data_as(ctypes.POINTER(ctypes.c_float)))
+    if r != 0:
+        raise ValueError("orc_swiglu_quantize: I must be a multiple of 128")
+    return q, sa, y
 
 
 def bf16_rne(x: float) -> int:

@@ -159,6 +159,55 @@ int orc_quantize_1x128(const uint16_t *x, int64_t M, int64_t K, uint8_t *q, floa
     return 0;
 }
 
+/* ---- SwiGLU followed by the per-token FP8 quantisation --------------------------------- */
+
+/* Between the two grouped GEMMs of an MoE layer (the fused gate/up projection, then the down
+ * projection; DeepGEMM release write-up, "如何使用": grouped GEMMs for MoE), each token row of
+ * the first GEMM's bf16 output h [M][2I] holds the gate half h[:, 0:I] and the up half
+ * h[:, I:2I].  The activation is
+ *     y[m][i] = silu(g) * u,  silu(g) = g / (1 + exp(-g)),  g = h[m][i], u = h[m][I + i]
+ * computed here in fp64 and rounded once to fp32 (y32, returned for the tests), then
+ * quantised exactly as orc_quantize_1x128 does (fp32 amax, factor 448 / amax, scale amax / 448,
+ * e4m3 round to nearest even).  Rows with row_valid[m] == 0 (NULL: all valid) are skipped and
+ * their outputs left untouched.  q [M][I], sa [M][I/128], y32 [M][I] (may be NULL). */
+int orc_swiglu_quantize(const uint16_t *h, int64_t M, int64_t I, const uint8_t *row_valid,
+                        uint8_t *q, float *sa, float *y32)
+{
+    if (I % ORC_BLOCK != 0 || M < 0)
+        return -1;
+    const int64_t kbs = I / ORC_BLOCK;
+    for (int64_t m = 0; m < M; ++m) {
+        if (row_valid && !row_valid[m])
+            continue;
+        for (int64_t kb = 0; kb < kbs; ++kb) {
+            float vals[ORC_BLOCK];
+            float amax = 0.0f;
+            for (int i = 0; i < ORC_BLOCK; ++i) {
+                const int64_t col = kb * ORC_BLOCK + i;
+                uint32_t wg = (uint32_t)h[m * 2 * I + col] << 16;
+                uint32_t wu = (uint32_t)h[m * 2 * I + I + col] << 16;
+                float g, u;
+                memcpy(&g, &wg, 4);
+                memcpy(&u, &wu, 4);
+                const double y = (double)g / (1.0 + exp(-(double)g)) * (double)u;
+                const float yf = (float)y;
+                vals[i] = yf;
+                if (y32)
+                    y32[m * I + col] = yf;
+                const float a = fabsf(yf);
+                if (a > amax)
+                    amax = a;
+            }
+            const float amax_c = amax > 1e-4f ? amax : 1e-4f;
+            const float factor = 448.0f / amax_c;
+            sa[m * kbs + kb] = amax_c / 448.0f;
+            for (int i = 0; i < ORC_BLOCK; ++i)
+                q[m * I + kb * ORC_BLOCK + i] = orc_e4m3_encode(vals[i] * factor);
+        }
+    }
+    return 0;
+}
+
 /* ---- one output row ------------------------------------------------------------------ */
 
 typedef struct {
