@@ -522,22 +522,27 @@ def run_reference(args):
     """The CPU oracle on a bounded sample of the workload (rank 0 only)."""
     import oracle
     oracle.build()
-    if args.workload == "quant":
-        M, K = args.shape[:2] if args.shape else (8192, 7168)
+    if args.workload in ("quant", "swiglu"):
+        swiglu = args.workload == "swiglu"
+        M, K = args.shape[:2] if args.shape else ((16384, 2048) if swiglu else (8192, 7168))
         rows = min(M, 256)
-        bits = quant_input(M, K)[:rows]
+        bits = quant_input(M, 2 * K if swiglu else K)[:rows]
+        fn = oracle.swiglu_quantize if swiglu else oracle.quantize_1x128
         for _ in range(args.warmup):
-            oracle.quantize_1x128(bits)
+            fn(bits)
         t0 = time.perf_counter()
         for _ in range(args.steps):
-            oracle.quantize_1x128(bits)
+            fn(bits)
         dt = time.perf_counter() - t0
-        value = args.steps * quant_bytes(rows, K) / dt / 1e9
+        value = args.steps * (swiglu_bytes(rows, K) if swiglu else quant_bytes(rows, K)) / dt / 1e9
         sample = f"the first {rows} rows per step"
-        return dict(metric=QUANT_METRIC, value=value, unit="GB/s", n_gpus=1, steps=args.steps,
+        wl = (f"SwiGLU + per-token FP8 quantisation M={M} I={K}" if swiglu
+              else f"per-token FP8 quantisation M={M} K={K}")
+        return dict(metric=SWIGLU_METRIC if swiglu else QUANT_METRIC, value=value, unit="GB/s",
+                    n_gpus=1, steps=args.steps,
                     warmup=args.warmup, ms_per_step=dt / args.steps * 1e3, higher_is_better=True,
                     scaling="weak", vs_baseline=None, dtype="f32", data="synthetic",
-                    config=dict(workload=f"per-token FP8 quantisation M={M} K={K}"), impl="reference",
+                    config=dict(workload=wl), impl="reference",
                     cpu_baseline=dict(value=value, unit="GB/s", cores=1, kind="oracle", sample=sample),
                     e2e=dict(value=value, unit="GB/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
     gemms, desc = build_workload(args.workload, args.shape)
@@ -580,14 +585,36 @@ def quant_bytes(M: int, K: int) -> float:
     return 2.0 * M * K + M * K + 4.0 * M * (K // 128)
 
 
+SWIGLU_METRIC = ("GB/s of SwiGLU + per-token FP8 quantisation (bf16 gate|up [M, 2I] -> e4m3 [M, I] + "
+                 "fp32 1x128 scales) at 1 B200; fraction of the HBM roofline")
+
+
+def swiglu_bytes(M: int, I: int) -> float:
+    return 2.0 * M * 2 * I + M * I + 4.0 * M * (I // 128)
+
+
 def run_quant(args, rank, world, local_rank):
+    """--workload quant: the per-token quantisation of an M x K activation (default 8192 x 7168);
+    --workload swiglu: SwiGLU + quantisation of an M x 2I gate|up tensor (default 16384 x 2*2048,
+    the per-expert intermediate width of DeepSeek-V3's MoE)."""
     import fp8_block_scaled_tma_b200 as dg
     torch.cuda.set_device(local_rank)
-    M, K = args.shape[:2] if args.shape else (8192, 7168)
-    bits = quant_input(M, K)
+    swiglu = args.workload == "swiglu"
+    if swiglu:
+        M, K = args.shape[:2] if args.shape else (16384, 2048)  # K = I
+        bits = quant_input(M, 2 * K)
+    else:
+        M, K = args.shape[:2] if args.shape else (8192, 7168)
+        bits = quant_input(M, K)
     x = torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
     q = torch.empty(M, K, dtype=torch.uint8, device="cuda")
     sfa = torch.empty(K // 128, dg.get_tma_aligned_size(M, 4), dtype=torch.float32, device="cuda")
+
+    def run_kernel():
+        if swiglu:
+            dg.swiglu_quantize_fp8_1x128(x, None, 0, q, sfa)
+        else:
+            dg.quantize_fp8_1x128(x, q, sfa)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -596,7 +623,7 @@ def run_quant(args, rank, world, local_rank):
         torch.cuda._sleep(200_000)
         flush.fill_(1)
         e0.record(stream)
-        dg.quantize_fp8_1x128(x, q, sfa)
+        run_kernel()
         e1.record(stream)
         stream.synchronize()
         return e0.elapsed_time(e1) * 1e-3
@@ -612,14 +639,16 @@ def run_quant(args, rank, world, local_rank):
     if dg.poll_device_error(stream) != 0:
         raise RuntimeError("device error")
     total = max_over_ranks(sum(ts), world, "cuda")
-    nbytes = quant_bytes(M, K)
+    nbytes = swiglu_bytes(M, K) if swiglu else quant_bytes(M, K)
     value = world * nbytes * args.steps / total / 1e9
     peaks = load_peaks()
     per = statistics.mean(ts)
     achieved = nbytes / per / 1e9
     roof = dict(bound="hbm", achieved=achieved, peak=peaks["hbm_gbs"], unit="GB/s",
                 frac=achieved / peaks["hbm_gbs"], frac_spec=achieved / SPEC_HBM_GBS,
-                peak_source=f"{peaks['source']} HBM copy", kernel=f"dg_quantize_1x128_kernel {M}x{K}",
+                peak_source=f"{peaks['source']} HBM copy",
+                kernel=(f"dg_swiglu_quantize_1x128_kernel {M}x{2 * K}" if swiglu
+                        else f"dg_quantize_1x128_kernel {M}x{K}"),
                 traffic=args.traffic_bytes, traffic_unit="bytes/launch")
     # e2e: pinned host bf16 in, quantise, codes and scales out
     hx = x.cpu().pin_memory()
@@ -629,7 +658,7 @@ def run_quant(args, rank, world, local_rank):
     def e2e_step():
         e0.record(stream)
         x.copy_(hx, non_blocking=True)
-        dg.quantize_fp8_1x128(x, q, sfa)
+        run_kernel()
         hq.copy_(q, non_blocking=True)
         hs.copy_(sfa, non_blocking=True)
         e1.record(stream)
@@ -639,12 +668,15 @@ def run_quant(args, rank, world, local_rank):
     e2e_step()
     et = [e2e_step() for _ in range(5)]
     e2e_t = max_over_ranks(sum(et), world, "cuda")
-    out = dict(metric=QUANT_METRIC, value=value, unit="GB/s", n_gpus=world, steps=args.steps,
+    out = dict(metric=SWIGLU_METRIC if swiglu else QUANT_METRIC, value=value, unit="GB/s",
+               n_gpus=world, steps=args.steps,
                warmup=args.warmup, ms_per_step=total / args.steps * 1e3, higher_is_better=True,
                scaling="weak", vs_baseline=None, dtype="bf16 -> e4m3 (fp32 arithmetic)",
                data="synthetic",
-               config=dict(workload=f"per-token FP8 quantisation M={M} K={K}, N(0,1) with 1% x50 outliers",
-                           l2="256 MiB write before every launch; input + output 176 MB > L2"),
+               config=dict(workload=(f"SwiGLU + per-token FP8 quantisation M={M} I={K}" if swiglu
+                                     else f"per-token FP8 quantisation M={M} K={K}")
+                                    + ", N(0,1) with 1% x50 outliers",
+                           l2=f"256 MiB write before every launch; input + output {nbytes / 1e6:.0f} MB > L2"),
                roofline=roof, gpu_launches=args.steps, clocks=clk.summary(),
                e2e=dict(value=world * nbytes * 5 / e2e_t / 1e9, unit="GB/s",
                         h2d_bytes_per_step=hx.numel() * 2, d2h_bytes_per_step=hq.numel() + hs.numel() * 4))
@@ -655,10 +687,14 @@ def run_quant(args, rank, world, local_rank):
         t0 = time.perf_counter()
         passes = 0
         while time.perf_counter() - t0 < min(args.cpu_seconds, 5.0):
-            oracle.quantize_1x128(bits[:rows])
+            if swiglu:
+                oracle.swiglu_quantize(bits[:rows])
+            else:
+                oracle.quantize_1x128(bits[:rows])
             passes += 1
         dt = time.perf_counter() - t0
-        out["cpu_baseline"] = dict(value=passes * quant_bytes(rows, K) / dt / 1e9, unit="GB/s", cores=1,
+        per_pass = swiglu_bytes(rows, K) if swiglu else quant_bytes(rows, K)
+        out["cpu_baseline"] = dict(value=passes * per_pass / dt / 1e9, unit="GB/s", cores=1,
                                    kind="oracle", sample=f"{passes} pass(es) over the first {rows} rows")
     return out
 
@@ -672,9 +708,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["sweep", "small", "contiguous", "masked", "prefill",
-                                           "dense", "quant"], default="sweep")
+                                           "dense", "quant", "swiglu"], default="sweep")
     ap.add_argument("--shape", type=lambda v: tuple(int(x) for x in v.split(",")), default=None,
-                    help="M,N,K of --workload dense; M,K of --workload quant")
+                    help="M,N,K of --workload dense; M,K of --workload quant; M,I of --workload swiglu")
     ap.add_argument("--block-n", type=int, default=0, help="tile override (tuning)")
     ap.add_argument("--stages", type=int, default=0, help="pipeline-stage override (tuning)")
     ap.add_argument("--splits", type=int, default=0, help="split-K override (tuning)")
@@ -707,7 +743,7 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        out = (run_quant if args.workload == "quant" else run_ours)(args, rank, world, local_rank)
+        out = (run_quant if args.workload in ("quant", "swiglu") else run_ours)(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(out), flush=True)
     finally:

@@ -74,6 +74,8 @@ def _load() -> ctypes.CDLL:
     lib.dg_set_kernel_family.argtypes = [i]
     lib.dg_set_kernel_family.restype = i
     lib.dg_quantize_fp8_1x128.argtypes = [vp, vp, fp, i, i, vp]
+    lib.dg_swiglu_quantize_fp8_1x128.argtypes = [vp, vp, fp, i, i, ip, i, vp]
+    lib.dg_swiglu_quantize_fp8_1x128.restype = i
     lib.dg_quantize_fp8_1x128.restype = i
     lib.dg_set_pdl.argtypes = [i]
     lib.dg_set_pdl.restype = i
@@ -267,6 +269,37 @@ def quantize_fp8_1x128(x, q=None, sfa=None, stream=None):
     _f32(sfa, "sfa", (K // BLOCK, get_tma_aligned_size(M, 4)))
     _check(lib.dg_quantize_fp8_1x128(_ptr(x), _ptr(q), _ptr(sfa), M, K, _stream(stream)),
            "dg_quantize_fp8_1x128")
+    return q, sfa
+
+
+def swiglu_quantize_fp8_1x128(h, masked_m=None, rows_per_group=0, q=None, sfa=None, stream=None):
+    """SwiGLU (gate half, then up half of each row of h bf16 [M, 2I]) followed by the per-token
+    FP8 quantisation.  Returns (q uint8 [M, I], sfa fp32): [I/128, align4(M)] without masked_m,
+    [G, I/128, align4(rows_per_group)] with it (the masked GEMM's layout)."""
+    if h.dtype != torch.bfloat16 or not h.is_cuda or not h.is_contiguous() or h.dim() != 2:
+        raise ValueError("h must be a contiguous 2-D bfloat16 CUDA tensor")
+    M, two_i = h.shape
+    I = two_i // 2
+    if two_i % 2 or I % BLOCK:
+        raise ValueError("h must be [M, 2I] with I a multiple of 128")
+    if q is None:
+        q = torch.empty(M, I, dtype=torch.uint8, device=h.device)
+    _fp8(q, "q")
+    if masked_m is not None:
+        if rows_per_group <= 0 or M % rows_per_group:
+            raise ValueError("rows_per_group must divide M")
+        G = M // rows_per_group
+        if masked_m.dtype != torch.int32 or tuple(masked_m.shape) != (G,) or not masked_m.is_cuda:
+            raise ValueError("masked_m must be an int32 CUDA tensor of G entries")
+        shape = (G, I // BLOCK, get_tma_aligned_size(rows_per_group, 4))
+    else:
+        shape = (I // BLOCK, get_tma_aligned_size(M, 4))
+    if sfa is None:
+        sfa = torch.empty(shape, dtype=torch.float32, device=h.device)
+    _f32(sfa, "sfa", shape)
+    _check(lib.dg_swiglu_quantize_fp8_1x128(_ptr(h), _ptr(q), _ptr(sfa), M, I, _ptr(masked_m),
+                                            int(rows_per_group), _stream(stream)),
+           "dg_swiglu_quantize_fp8_1x128")
     return q, sfa
 
 

@@ -925,6 +925,38 @@ int check_common(const void *a, const float *sfa, const void *b, const float *sf
     return DG_OK;
 }
 
+int launch_swiglu_quantize(const void *h, void *q, float *sfa, int M, int I, const int *masked_m,
+                           int rows_per_group, void *stream)
+{
+    int dev = 0;
+    DeviceInfo *info = nullptr;
+    int st = device_setup(dev, info);
+    if (st != DG_OK)
+        return st;
+    const long long blocks_x = (static_cast<long long>(M) + dg::kQuantRowsPerBlock - 1) / dg::kQuantRowsPerBlock;
+    if (blocks_x > 0x7FFFFFFFLL || I / dg::kBlockK > 65535)
+        return DG_ERR_INVALID_ARG;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(static_cast<unsigned>(blocks_x), static_cast<unsigned>(I / dg::kBlockK), 1);
+    cfg.blockDim = dim3(dg::kQuantThreads, 1, 1);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    cfg.attrs = attr;
+    cfg.numAttrs = add_pdl_attr(attr, 0);
+    const __nv_bfloat16 *hp = static_cast<const __nv_bfloat16 *>(h);
+    uint8_t *qp = static_cast<uint8_t *>(q);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, dg::dg_swiglu_quantize_1x128_kernel, hp, qp, sfa, M, I,
+                                       masked_m, rows_per_group);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        if (debug_enabled())
+            std::fprintf(stderr, "[dg] swiglu-quantize launch failed: %s\n", cudaGetErrorString(e));
+        return DG_ERR_CUDA;
+    }
+    return DG_OK;
+}
+
 int launch_quantize(const void *x, void *q, float *sfa, int M, int K, void *stream)
 {
     int dev = 0;
@@ -960,6 +992,20 @@ int launch_quantize(const void *x, void *q, float *sfa, int M, int K, void *stre
 }  // namespace
 
 extern "C" {
+
+int dg_swiglu_quantize_fp8_1x128(const void *h, void *q, float *sfa, int M, int I,
+                                 const int *masked_m, int rows_per_group, void *stream)
+{
+    if (M < 0 || I <= 0 || I % dg::kBlockK != 0)
+        return DG_ERR_INVALID_ARG;
+    if (masked_m != nullptr && (rows_per_group <= 0 || M % rows_per_group != 0))
+        return DG_ERR_INVALID_ARG;
+    if (M == 0)
+        return DG_OK;
+    if (!h || !q || !sfa || !aligned16(h) || !aligned16(q) || !aligned16(sfa))
+        return DG_ERR_INVALID_ARG;
+    return launch_swiglu_quantize(h, q, sfa, M, I, masked_m, masked_m ? rows_per_group : 0, stream);
+}
 
 int dg_quantize_fp8_1x128(const void *x, void *q, float *sfa, int M, int K, void *stream)
 {

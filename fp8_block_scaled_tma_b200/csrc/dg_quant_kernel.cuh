@@ -127,4 +127,97 @@ __global__ void __launch_bounds__(kQuantThreads)
     }
 }
 
+// ---- SwiGLU followed by the same quantisation --------------------------------------------------
+// Between the two grouped GEMMs of an MoE layer: each row of the first GEMM's bf16 output h
+// [M][2I] holds the gate half h[:, 0:I] and the up half h[:, I:2I]; the second GEMM's A operand
+// is y = silu(gate) * up, silu(g) = g / (1 + exp(-g)) in fp32 with the GPU's fast exponential
+// and division (y within a few fp32 ulps of exact), quantised per 1 x 128 tile as above.  With masked_m (the masked MoE layout, M = G * rows_per_group), row r of group g is
+// processed only when r < masked_m[g], and the scales use that layout's per-group form
+// [G][I/128][align4(rows_per_group)]; otherwise all rows, scales [I/128][align4(M)].
+__global__ void __launch_bounds__(kQuantThreads)
+    dg_swiglu_quantize_1x128_kernel(const __nv_bfloat16 *__restrict__ h, uint8_t *__restrict__ q,
+                                    float *__restrict__ sfa, int M, int I, const int *masked_m,
+                                    int rows_per_group)
+{
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();
+    const int lane = threadIdx.x & 31;
+    const int half = lane >> 4;
+    const int hl = lane & 15;
+    const int kb = blockIdx.y;
+    const int kbs = I / 128;
+    const int row0 = blockIdx.x * kQuantRowsPerBlock + (threadIdx.x >> 5) * kQuantRowsPerWarp;
+    const size_t col = static_cast<size_t>(kb) * 128 + hl * 8;
+    bool valid[kQuantUnroll];
+    uint4 gr[kQuantUnroll], ur[kQuantUnroll];
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+        const int row = row0 + 2 * u + half;
+        bool v = row < M;
+        if (v && masked_m != nullptr) {
+            const int g = row / rows_per_group;
+            v = row - g * rows_per_group < __ldg(masked_m + g);
+        }
+        valid[u] = v;
+        if (v) {
+            const __nv_bfloat16 *hr = h + static_cast<size_t>(row) * 2 * I + col;
+            gr[u] = ld_nc_v4(hr);
+            ur[u] = ld_nc_v4(hr + I);
+        } else {
+            gr[u] = make_uint4(0, 0, 0, 0);
+            ur[u] = make_uint4(0, 0, 0, 0);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) {
+        const int row = row0 + 2 * u + half;
+        const uint32_t gw[4] = {gr[u].x, gr[u].y, gr[u].z, gr[u].w};
+        const uint32_t uw[4] = {ur[u].x, ur[u].y, ur[u].z, ur[u].w};
+        float y[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const float g = __uint_as_float(j == 0 ? gw[i] << 16 : gw[i] & 0xFFFF0000u);
+                const float up = __uint_as_float(j == 0 ? uw[i] << 16 : uw[i] & 0xFFFF0000u);
+                // fast exponential and division (a few ulps; 0 for 1 + e^-g beyond 2^126,
+                // the limit of silu there)
+                y[2 * i + j] = __fdividef(g, 1.0f + __expf(-g)) * up;
+            }
+        }
+        float amax = fabsf(y[0]);
+#pragma unroll
+        for (int i = 1; i < 8; ++i)
+            amax = fmaxf(amax, fabsf(y[i]));
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1)  // within the half-warp of this row
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        amax = fmaxf(amax, 1e-4f);
+        const float factor = 448.0f / amax;
+        const float scale = amax / 448.0f;
+        if (valid[u]) {
+            const uint32_t c01 = cvt_e4m3x2(y[0] * factor, y[1] * factor);
+            const uint32_t c23 = cvt_e4m3x2(y[2] * factor, y[3] * factor);
+            const uint32_t c45 = cvt_e4m3x2(y[4] * factor, y[5] * factor);
+            const uint32_t c67 = cvt_e4m3x2(y[6] * factor, y[7] * factor);
+            uint2 out;
+            out.x = c01 | (c23 << 16);
+            out.y = c45 | (c67 << 16);
+            *reinterpret_cast<uint2 *>(q + static_cast<size_t>(row) * I + col) = out;
+            if (hl == 0) {
+                size_t idx;
+                if (masked_m != nullptr) {
+                    const int g = row / rows_per_group;
+                    const int r = row - g * rows_per_group;
+                    const int ld = (rows_per_group + 3) / 4 * 4;
+                    idx = (static_cast<size_t>(g) * kbs + kb) * ld + r;
+                } else {
+                    idx = static_cast<size_t>(kb) * ((M + 3) / 4 * 4) + row;
+                }
+                sfa[idx] = scale;
+            }
+        }
+    }
+}
+
 }  // namespace dg

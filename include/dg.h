@@ -110,6 +110,28 @@ int dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked(const void *a, const float *sfa, co
  * Returns DG_OK, DG_ERR_INVALID_ARG (nothing launched), DG_ERR_UNSUPPORTED or DG_ERR_CUDA. */
 int dg_quantize_fp8_1x128(const void *x, void *q, float *sfa, int M, int K, void *stream);
 
+/* SwiGLU followed by the same per-token FP8 quantisation: the step between the two grouped
+ * GEMMs of an MoE layer ("如何使用": grouped GEMMs for MoE; the fused gate/up projection's bf16
+ * output feeds the down projection's FP8 A operand).  Row m of h holds the gate half h[m][0:I]
+ * and the up half h[m][I:2I]; in fp32
+ *     y[m][i] = silu(g) * u,  silu(g) = g / (1 + exp(-g)),  g = h[m][i], u = h[m][I + i]
+ * and y is quantised per 1 x 128 tile exactly as dg_quantize_fp8_1x128 does.
+ *   h         bf16 [M][2I] row-major (device)
+ *   q         e4m3 codes [M][I] row-major (device, written for processed rows)
+ *   sfa       fp32 scales: without masked_m [I/128][align4(M)] (the dense / contiguous
+ *             layout); with masked_m [G][I/128][align4(rows_per_group)] (the masked layout),
+ *             G = M / rows_per_group
+ *   masked_m  NULL (every row) or int32 [G] on the device: row r of group g (r = m mod
+ *             rows_per_group) is processed only when r < masked_m[g]; other rows' q and sfa
+ *             entries are not written
+ *   M >= 0, I > 0 and I % 128 == 0, I/128 <= 65535, pointers 16-byte aligned; with masked_m,
+ *   rows_per_group > 0 and M % rows_per_group == 0.  exp is the GPU's fast exponential, so y
+ * can differ from an exact evaluation by a few fp32 ulps (codes can then differ by one step
+ *   next to an e4m3 rounding midpoint).  Returns DG_OK, DG_ERR_INVALID_ARG (nothing
+ *   launched), DG_ERR_UNSUPPORTED or DG_ERR_CUDA. */
+int dg_swiglu_quantize_fp8_1x128(const void *h, void *q, float *sfa, int M, int I,
+                                 const int *masked_m, int rows_per_group, void *stream);
+
 /* The SM-count utility of "如何使用": caps the number of SMs the persistent kernels occupy so
  * that other work (for example communication kernels) can run beside them.  n <= 0 restores
  * "all SMs".  Returns the previous cap (0 = all). */

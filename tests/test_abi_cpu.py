@@ -22,8 +22,8 @@ def declared_functions():
 
 @pytest.fixture(scope="module")
 def dg():
-    from fp8_block_scaled_tma_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__._library_builder().build()
     import fp8_block_scaled_tma_b200 as mod
     return mod
 
