@@ -276,18 +276,17 @@ __device__ __forceinline__ bool promote_kb(float (&acc)[NCOLS], float sa, float 
 
 // The K loop of a promotion thread for one tile.  It is unrolled by two with two named scale
 // sets, each reloaded right after its use, so a scale load has a whole K block to land and no
-// register move waits on it.  `tbuf_release(buf)` gives the barrier address that frees buffer
-// `buf` (and whether it is remote).
+// register move waits on it.  s0 / s1 arrive holding the scales of K blocks 0 and 1 (loaded by
+// the caller, early enough to have landed).  `tbuf_release(buf)` gives the barrier address that
+// frees buffer `buf` (and whether it is remote).
 template <int BN, int P1, int P2, int NCOLS, int NBUF, class Release>
-__device__ __forceinline__ bool promote_tile(float (&acc)[NCOLS], const float *sa_ptr,
-                                             const float *sb_lo, const float *sb_hi,
-                                             uint32_t lane_base, uint32_t bar_tfull, int &buf,
-                                             uint32_t &bph, Release tbuf_release, int split,
-                                             int lane, const Params &p, volatile int *abort_flag)
+__device__ __forceinline__ bool promote_tile(float (&acc)[NCOLS], KbScales s0, KbScales s1,
+                                             const float *sa_ptr, const float *sb_lo,
+                                             const float *sb_hi, uint32_t lane_base,
+                                             uint32_t bar_tfull, int &buf, uint32_t &bph,
+                                             Release tbuf_release, int split, int lane,
+                                             const Params &p, volatile int *abort_flag)
 {
-    KbScales s0, s1;
-    load_kb_scales(s0, sa_ptr, sb_lo, sb_hi, p.sfa_ld, 0, p.num_kb);
-    load_kb_scales(s1, sa_ptr, sb_lo, sb_hi, p.sfa_ld, 1, p.num_kb);
     auto step = [&](const KbScales &sc) -> bool {
         uint32_t rel;
         bool remote;
@@ -702,39 +701,61 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         int buf = 0;
         uint32_t bph = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        // Everything a thread needs to start a tile, including the scales of its first two K
+        // blocks: prepared for the next tile before the current tile's epilogue, so that those
+        // global loads land while the epilogue runs instead of stalling the first promotion.
+        struct TileCtx {
             Tile ti;
-            if (!resolve_tile<L>(p, ctl, t, ti))
-                continue;
-            const int n0 = ti.n0 * BN;
-            const int col0 = n0 + half * C::kCols;  // first global column of this thread
+            int col0, split;
+            const float *sfb_lo, *sfb_hi, *sa_ptr;
+            KbScales s0, s1;
+        };
+        auto prepare = [&](int t, TileCtx &c) -> bool {
+            if (!resolve_tile<L>(p, ctl, t, c.ti))
+                return false;
+            c.col0 = c.ti.n0 * BN + half * C::kCols;  // first global column of this thread
             // the (at most two) 128-column scale blocks of B this thread's columns touch; the
             // boundary (if any) lies on a 16-column group edge
-            const int nb_lo = min(col0 / kBlockK, p.num_nb - 1);
-            const int nb_hi = min((col0 + C::kCols - 1) / kBlockK, p.num_nb - 1);
-            const int split = min(C::kCols, max(0, (nb_lo + 1) * kBlockK - col0));  // first hi column
-            const float *sfb_lo = p.sfb + (static_cast<size_t>(ti.g) * p.num_nb + nb_lo) * p.num_kb;
-            const float *sfb_hi = p.sfb + (static_cast<size_t>(ti.g) * p.num_nb + nb_hi) * p.num_kb;
-            // this thread's A scales: one per K block, num_kb rows of sfa_ld apart (rows past the
-            // scale matrix read its last row; they are not stored)
-            const float *sa_ptr = p.sfa + static_cast<size_t>(ti.a_z) * p.num_kb * p.sfa_ld +
-                                  min(ti.m0 + row, p.sfa_ld - 1);
-
+            const int nb_lo = min(c.col0 / kBlockK, p.num_nb - 1);
+            const int nb_hi = min((c.col0 + C::kCols - 1) / kBlockK, p.num_nb - 1);
+            c.split = min(C::kCols, max(0, (nb_lo + 1) * kBlockK - c.col0));  // first hi column
+            c.sfb_lo = p.sfb + (static_cast<size_t>(c.ti.g) * p.num_nb + nb_lo) * p.num_kb;
+            c.sfb_hi = p.sfb + (static_cast<size_t>(c.ti.g) * p.num_nb + nb_hi) * p.num_kb;
+            // this thread's A scales: one per K block, num_kb rows of sfa_ld apart (rows past
+            // the scale matrix read its last row; they are not stored)
+            c.sa_ptr = p.sfa + static_cast<size_t>(c.ti.a_z) * p.num_kb * p.sfa_ld +
+                       min(c.ti.m0 + row, p.sfa_ld - 1);
+            load_kb_scales(c.s0, c.sa_ptr, c.sfb_lo, c.sfb_hi, p.sfa_ld, 0, p.num_kb);
+            load_kb_scales(c.s1, c.sa_ptr, c.sfb_lo, c.sfb_hi, p.sfa_ld, 1, p.num_kb);
+            return true;
+        };
+        int t = blockIdx.x;
+        TileCtx cur;
+        while (t < num_tiles && !prepare(t, cur))
+            t += gridDim.x;
+        while (t < num_tiles && ok) {
+            const Tile ti = cur.ti;
+            const int col0 = cur.col0;
             float acc[C::kCols];
 #pragma unroll
             for (int c = 0; c < C::kCols; ++c)
                 acc[c] = 0.0f;
 
-            // scales of K blocks kb (cur) and kb + 1 (nxt) are in registers; kb + 2 is loaded
             ok = promote_tile<BN, P1, P2, C::kCols, C::kTmemBufs>(
-                acc, sa_ptr, sfb_lo, sfb_hi, lane_base, bar_tfull, buf, bph,
+                acc, cur.s0, cur.s1, cur.sa_ptr, cur.sfb_lo, cur.sfb_hi, lane_base, bar_tfull, buf,
+                bph,
                 [&](int b, uint32_t &rel, bool &remote) {
                     rel = bar_tempty + 8 * b;
                     remote = false;
                 },
-                split, lane, p, abort_flag);
+                cur.split, lane, p, abort_flag);
             if (!ok)
                 break;
+            // the next tile of this CTA, its scales in flight during this epilogue
+            int tn = t + static_cast<int>(gridDim.x);
+            while (tn < num_tiles && !prepare(tn, cur))
+                tn += gridDim.x;
+            t = tn;
 
             // ---- epilogue: bf16 rounding, TMA stores of whole warps, direct stores otherwise ----
             const int grow = ti.m0 + row;  // row within the group

@@ -263,8 +263,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         uint32_t bph = 0;
         Params pk = p;
         pk.num_kb = nkb;  // the promotion loop walks this CTA's K blocks only
+        KbScales s0, s1;
+        load_kb_scales(s0, sa_ptr, sfb_lo, sfb_hi, p.sfa_ld, 0, nkb);
+        load_kb_scales(s1, sa_ptr, sfb_lo, sfb_hi, p.sfa_ld, 1, nkb);
         promote_tile<BN, P1, P2, C::kCols, C::kTmemBufs>(
-            acc, sa_ptr, sfb_lo, sfb_hi, lane_base, bar_tfull, buf, bph,
+            acc, s0, s1, sa_ptr, sfb_lo, sfb_hi, lane_base, bar_tfull, buf, bph,
             [&](int b, uint32_t &rel, bool &remote) {
                 rel = bar_tempty + 8 * b;
                 remote = false;
