@@ -46,6 +46,16 @@ FP8_PER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor ratio on B200 (4.5 / 2.25 
 SPEC_FP8_TFLOPS = 4500.0  # B200 dense FP8 tensor peak (data sheet)
 SPEC_HBM_GBS = 8000.0     # B200 HBM3e bandwidth (data sheet)
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernel
+# of each default workload, from one ncu capture of the current kernels (summaries under
+# profiles/).  `roofline.traffic` reports it; --traffic-bytes overrides it.  Re-measure after a
+# kernel change (a stale figure is worse than none).
+MEASURED_TRAFFIC = {
+    "dense 4096x7168x16384": 487783424 + 53111808,            # CTA pair BN 224
+    "dg_quantize_1x128_kernel 8192x7168": 117451520 + 9024512,
+    "dg_swiglu_quantize_1x128_kernel 16384x4096": 134243072 + 7325696,
+}
+
 
 # ---- workload description ---------------------------------------------------------------------
 
@@ -416,7 +426,9 @@ def run_ours(args, rank, world, local_rank):
         peak = peaks["hbm_gbs"]
         roof = dict(bound="hbm", achieved=dsh["gbs"], peak=peak, unit="GB/s",
                     frac=dsh["gbs"] / peak, peak_source=f"{peaks['source']} HBM copy")
-    roof.update(kernel=dsh["name"], traffic=args.traffic_bytes, traffic_unit="bytes/launch",
+    roof.update(kernel=dsh["name"],
+                traffic=args.traffic_bytes if args.traffic_bytes else MEASURED_TRAFFIC.get(dsh["name"]),
+                traffic_unit="bytes/launch",
                 frac_spec=dsh["frac_spec"])
     if rank == 0 and not args.no_cublas:
         # context only: what cuBLAS reaches on an FP8 GEMM on this GPU
@@ -649,7 +661,8 @@ def run_quant(args, rank, world, local_rank):
                 peak_source=f"{peaks['source']} HBM copy",
                 kernel=(f"dg_swiglu_quantize_1x128_kernel {M}x{2 * K}" if swiglu
                         else f"dg_quantize_1x128_kernel {M}x{K}"),
-                traffic=args.traffic_bytes, traffic_unit="bytes/launch")
+                traffic_unit="bytes/launch")
+    roof["traffic"] = args.traffic_bytes if args.traffic_bytes else MEASURED_TRAFFIC.get(roof["kernel"])
     # e2e: pinned host bf16 in, quantise, codes and scales out
     hx = x.cpu().pin_memory()
     hq = torch.empty_like(q, device="cpu").pin_memory()
