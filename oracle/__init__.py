@@ -57,6 +57,11 @@ def _load():
                                         ctypes.POINTER(ctypes.c_uint8), ctypes.POINTER(ctypes.c_uint8),
                                         ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]
     lib.orc_swiglu_quantize.restype = ctypes.c_int
+    lib.orc_e2m1_decode.argtypes = [ctypes.c_uint8]
+    lib.orc_e2m1_decode.restype = ctypes.c_double
+    lib.orc_e2m1_to_e4m3.argtypes = [ctypes.POINTER(ctypes.c_uint8), ctypes.c_int64, ctypes.c_int64,
+                                     ctypes.POINTER(ctypes.c_uint8)]
+    lib.orc_e2m1_to_e4m3.restype = None
     lib.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
     lib.orc_e4m3_decode.restype = ctypes.c_double
     lib.orc_bf16_rne.argtypes = [ctypes.c_double]
@@ -131,6 +136,22 @@ def swiglu_quantize(h_bits: np.ndarray, row_valid: np.ndarray | None = None):
     if r != 0:
         raise ValueError("orc_swiglu_quantize: I must be a multiple of 128")
     return q, sa, y
+
+
+def e2m1_decode(nibble: int) -> float:
+    return float(_load().orc_e2m1_decode(int(nibble) & 0xF))
+
+
+def e2m1_to_e4m3(packed: np.ndarray) -> np.ndarray:
+    """Packed E2M1 [..., rows, K/2] (element 2j in the low nibble of byte j) -> E4M3 codes
+    [..., rows, K] of the same values."""
+    p = np.ascontiguousarray(packed, dtype=np.uint8)
+    lead, half_k = p.shape[:-1], p.shape[-1]
+    rows = int(np.prod(lead)) if lead else 1
+    out = np.empty(lead + (2 * half_k,), dtype=np.uint8)
+    _load().orc_e2m1_to_e4m3(p.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)), rows, 2 * half_k,
+                             out.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+    return out
 
 
 def bf16_rne(x: float) -> int:

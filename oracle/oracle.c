@@ -119,6 +119,29 @@ uint8_t orc_e4m3_encode(float v)
     return sign | (uint8_t)(code > 0x7E ? 0x7E : code);
 }
 
+/* OCP 4-bit floating point E2M1 (the FP4 of FP8 x FP4 GEMMs, the later DeepGEMM release, page
+ * 2): bit 3 the sign, bits 2..1 the exponent (bias 1), bit 0 the mantissa; exponent 0 is
+ * subnormal (m / 2).  Values +-{0, 0.5, 1, 1.5, 2, 3, 4, 6}; no infinities or NaN. */
+double orc_e2m1_decode(uint8_t nibble)
+{
+    const int s = (nibble >> 3) & 1, e = (nibble >> 1) & 3, m = nibble & 1;
+    const double mag = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -mag : mag;
+}
+
+/* Expands packed E2M1 rows (two elements per byte, element 2j in the low nibble of byte j)
+ * into E4M3 codes of the same values -- every E2M1 value is an E4M3 value -- so the FP8 x FP4
+ * GEMM is the FP8 GEMM of the expanded operand.  packed [rows][K/2] -> codes [rows][K]. */
+void orc_e2m1_to_e4m3(const uint8_t *packed, int64_t rows, int64_t K, uint8_t *codes)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < K; ++k) {
+            const uint8_t byte = packed[r * (K / 2) + k / 2];
+            const uint8_t nib = (k & 1) ? (byte >> 4) : (byte & 0xF);
+            codes[r * K + k] = orc_e4m3_encode((float)orc_e2m1_decode(nib));
+        }
+}
+
 /* ---- per-token (1 x 128) FP8 quantisation of bf16 activations ------------------------- */
 
 /* The step before the GEMM (DeepGEMM release write-up, "深入了解DeepGEMM": activations carry
