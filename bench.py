@@ -2,7 +2,8 @@
 """Benchmark of the FP8 block-scaled NT GEMM library on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload sweep|small|contiguous|masked|prefill]
+                    [--workload sweep|small|contiguous|masked|prefill|dense|quant|swiglu]
+                    [--fp4]
 
 Prints ONE JSON line on rank 0.  A "step" is one pass of the whole hot path over one batch of
 synthetic input: for the default workload, the fifteen GEMMs of the dense sweep
@@ -18,7 +19,8 @@ device times), summed over ranks (each rank runs its own copy of the step: weak 
 collective on the data path).  `e2e` is the same metric through the Python binding with host
 buffers: pinned host -> device copies of every input, the GEMMs, and the device -> host copy of
 every output inside the timed region.  `--impl reference` times the CPU oracle on a bounded
-sample of the same workload on this machine's cores.
+sample of the same workload on this machine's cores.  `--fp4` makes B of every GEMM a packed
+FP4 (E2M1) operand and runs the FP8 x FP4 entries on the same workload.
 """
 from __future__ import annotations
 
@@ -62,8 +64,9 @@ MEASURED_TRAFFIC = {
 class Gemm:
     """One GEMM of a step: its kind, sizes, FLOPs and algorithmic bytes."""
 
-    def __init__(self, kind: str, case, name: str):
-        self.kind, self.case, self.name = kind, case, name
+    def __init__(self, kind: str, case, name: str, fp4: bool = False):
+        self.kind, self.case, self.name, self.fp4 = kind, case, name, fp4
+        self._oracle_b = None
         c = case
         if kind == "dense":
             M, N, K, groups, m_valid, m_rows = c.M, c.N, c.K, 1, c.M, c.M
@@ -79,12 +82,36 @@ class Gemm:
         self.flops = 2.0 * m_valid * N * K
         # each operand once: A rows that are computed, B of every group touched, D, the scales,
         # and the int32 row indices of the contiguous layout
-        self.bytes = (m_valid * K + N * K * groups + 2 * m_valid * N + 4 * m_rows * kb
+        # (a packed FP4 B is half a byte per element)
+        b_bytes = N * K * groups // (2 if fp4 else 1)
+        self.bytes = (m_valid * K + b_bytes + 2 * m_valid * N + 4 * m_rows * kb
                       + 4 * nb * kb * groups + (4 * M if kind == "contiguous" else 0))
         self.shape = dict(kind=kind, M=M, N=N, K=K, G=getattr(c, "G", 1), M_valid=m_valid)
 
+    def oracle_b(self):
+        """B as the oracle takes it: e4m3 codes (an FP4 B expanded once by the oracle)."""
+        if not self.fp4:
+            return self.case.b
+        if self._oracle_b is None:
+            import oracle
+            self._oracle_b = oracle.e2m1_to_e4m3(self.case.b)
+        return self._oracle_b
 
-def build_workload(name: str, shape=None):
+
+def build_workload(name: str, shape=None, fp4: bool = False):
+    """The GEMMs of one step.  fp4: every B becomes a packed E2M1 operand (seeded, with its own
+    128x128 block scales) and the step runs the FP8 x FP4 entries."""
+    gemms, desc = _build_workload(name, shape)
+    if not fp4:
+        return gemms, desc
+    out = []
+    for i, g in enumerate(gemms):
+        out.append(Gemm(g.kind, workloads.with_fp4_b(g.case, seed=7000 + i), g.name + " fp4", fp4=True))
+    return out, desc.replace("B~N(0,0.02)", "B packed FP4 E2M1 (uniform codes, 128x128 fp32 block scales)") \
+        + "; FP8 x FP4"
+
+
+def _build_workload(name: str, shape=None):
     if name == "dense":
         M, N, K = shape
         c = workloads.dense(M, N, K, seed=6000, a_std=1.0, b_std=0.02)
@@ -330,7 +357,17 @@ class DeviceGemm:
 
     def launch(self, stream=None):
         dg, c = self.dg, self.g.case
-        if self.g.kind == "dense":
+        if self.g.fp4:
+            if self.g.kind == "dense":
+                dg.dg_gemm_fp8_fp4_bf16_nt(self.a, self.sfa, self.b, self.sfb, self.d, stream=stream)
+            elif self.g.kind == "contiguous":
+                dg.dg_m_grouped_gemm_fp8_fp4_bf16_nt_contiguous(self.a, self.sfa, self.b, self.sfb,
+                                                                self.d, self.extra, stream=stream)
+            else:
+                dg.dg_m_grouped_gemm_fp8_fp4_bf16_nt_masked(self.a, self.sfa, self.b, self.sfb,
+                                                            self.d, self.extra, c.expected_m,
+                                                            stream=stream)
+        elif self.g.kind == "dense":
             dg.dg_gemm_fp8_fp8_bf16_nt(self.a, self.sfa, self.b, self.sfb, self.d, stream=stream)
         elif self.g.kind == "contiguous":
             dg.dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(self.a, self.sfa, self.b, self.sfb,
@@ -344,7 +381,7 @@ def run_ours(args, rank, world, local_rank):
     import fp8_block_scaled_tma_b200 as dg
 
     torch.cuda.set_device(local_rank)
-    gemms, desc = build_workload(args.workload, args.shape)
+    gemms, desc = build_workload(args.workload, args.shape, args.fp4)
     if args.block_n or args.stages or args.splits:
         dg.set_config_override(args.block_n, args.stages, args.splits)
     if args.family:
@@ -436,7 +473,8 @@ def run_ours(args, rank, world, local_rank):
 
     out = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps,
                warmup=args.warmup, ms_per_step=total_max / args.steps * 1e3,
-               higher_is_better=True, scaling="weak", vs_baseline=None, dtype="e4m3 x e4m3 -> f32",
+               higher_is_better=True, scaling="weak", vs_baseline=None,
+               dtype="e4m3 x e2m1 -> f32" if args.fp4 else "e4m3 x e4m3 -> f32",
                data="synthetic",
                config=dict(workload=desc, gemms_per_step=n,
                            l2="256 MiB write before every step; step working set > L2 (126 MB)",
@@ -493,16 +531,16 @@ def _oracle_rows(g: Gemm, rows_per_gemm: int, rng):
     c = g.case
     if g.kind == "dense":
         r = np.sort(rng.choice(c.M, size=min(c.M, rows_per_gemm), replace=False))
-        oracle.gemm_dense(c.a, c.sa, c.b, c.sb, rows=r)
+        oracle.gemm_dense(c.a, c.sa, g.oracle_b(), c.sb, rows=r)
         return 2.0 * len(r) * c.N * c.K
     if g.kind == "contiguous":
         valid = np.nonzero(c.m_indices >= 0)[0]
         r = np.sort(rng.choice(valid, size=min(len(valid), rows_per_gemm), replace=False))
-        oracle.gemm_contiguous(c.a, c.sa, c.b, c.sb, c.m_indices, rows=r)
+        oracle.gemm_contiguous(c.a, c.sa, g.oracle_b(), c.sb, c.m_indices, rows=r)
         return 2.0 * len(r) * c.N * c.K
     flat = np.array([gi * c.M_max + r for gi in range(c.G) for r in range(int(c.masked_m[gi]))])
     r = np.sort(rng.choice(flat, size=min(len(flat), rows_per_gemm), replace=False))
-    oracle.gemm_masked(c.a, c.sa, c.b, c.sb, c.masked_m, rows=r)
+    oracle.gemm_masked(c.a, c.sa, g.oracle_b(), c.sb, c.masked_m, rows=r)
     return 2.0 * len(r) * c.N * c.K
 
 
@@ -518,6 +556,8 @@ def cpu_baseline(gemms, budget_s: float = 15.0):
     cores = os.cpu_count() or 1
     rows = max(16, cores)
     rng = np.random.default_rng(1234)
+    for g in gemms:
+        g.oracle_b()  # an FP4 B is expanded once, outside the timed sample
     flops, t0, passes = 0.0, time.perf_counter(), 0
     while True:
         flops += oracle_sample_step(gemms, rows, rng)
@@ -557,7 +597,9 @@ def run_reference(args):
                     config=dict(workload=wl), impl="reference",
                     cpu_baseline=dict(value=value, unit="GB/s", cores=1, kind="oracle", sample=sample),
                     e2e=dict(value=value, unit="GB/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
-    gemms, desc = build_workload(args.workload, args.shape)
+    gemms, desc = build_workload(args.workload, args.shape, args.fp4)
+    for g in gemms:
+        g.oracle_b()
     cores = os.cpu_count() or 1
     rows = 16
     rng = np.random.default_rng(99)
@@ -729,6 +771,8 @@ def main():
     ap.add_argument("--splits", type=int, default=0, help="split-K override (tuning)")
     ap.add_argument("--family", type=int, default=0,
                     help="kernel family override (tuning): 1 one-CTA, 2 CTA pair, 3 split-K")
+    ap.add_argument("--fp4", action="store_true",
+                    help="B of every GEMM as packed FP4 E2M1 (the FP8 x FP4 entries)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph timing of memory-bound shapes")
@@ -739,6 +783,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.fp4 and args.workload in ("quant", "swiglu"):
+        raise SystemExit("--fp4 applies to the GEMM workloads")
     if args.workload == "dense" and (args.shape is None or len(args.shape) != 3):
         raise SystemExit("--workload dense needs --shape M,N,K")
 

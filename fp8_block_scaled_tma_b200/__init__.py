@@ -50,8 +50,15 @@ def _load() -> ctypes.CDLL:
                                                                  i, vp, sz, vp]
     lib.dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked.argtypes = [vp, fp, vp, fp, vp, ip, i, i, i, i,
                                                              i, vp, sz, vp]
+    lib.dg_gemm_fp8_fp4_bf16_nt.argtypes = [vp, fp, vp, fp, vp, i, i, i, vp]
+    lib.dg_m_grouped_gemm_fp8_fp4_bf16_nt_contiguous.argtypes = [vp, fp, vp, fp, vp, ip, i, i, i,
+                                                                 i, vp]
+    lib.dg_m_grouped_gemm_fp8_fp4_bf16_nt_masked.argtypes = [vp, fp, vp, fp, vp, ip, i, i, i, i,
+                                                             i, vp]
     for name in ("dg_gemm_fp8_fp8_bf16_nt", "dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous",
-                 "dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked"):
+                 "dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked", "dg_gemm_fp8_fp4_bf16_nt",
+                 "dg_m_grouped_gemm_fp8_fp4_bf16_nt_contiguous",
+                 "dg_m_grouped_gemm_fp8_fp4_bf16_nt_masked"):
         getattr(lib, name).restype = ctypes.c_int
     lib.dg_set_num_sms.argtypes = [i]
     lib.dg_set_num_sms.restype = i
@@ -116,6 +123,16 @@ def _fp8(t: torch.Tensor, name: str) -> None:
         raise TypeError(f"{name} must hold e4m3 codes (uint8 or float8_e4m3fn), got {t.dtype}")
     if not t.is_cuda or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
+
+
+def _fp4(t: torch.Tensor, name: str) -> None:
+    fp4_x2 = getattr(torch, "float4_e2m1fn_x2", None)
+    if t.dtype != torch.uint8 and t.dtype != fp4_x2:
+        raise TypeError(f"{name} must hold packed e2m1 pairs (uint8 or float4_e2m1fn_x2), got {t.dtype}")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if t.data_ptr() % 32 != 0:
+        raise ValueError(f"{name} must be 32-byte aligned")
 
 
 def _f32(t: torch.Tensor, name: str, shape) -> None:
@@ -342,3 +359,58 @@ def dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked(a, sfa, b, sfb, d, masked_m, expect
         _ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), _ptr(masked_m), G, M_max, N, K,
         int(expected_m), _ptr(workspace), ws, _stream(stream)),
         "dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked")
+
+
+# ---- FP8 x FP4: b holds packed E2M1 pairs, [.., N, K/2] bytes, element 2j in the low nibble --
+
+def dg_gemm_fp8_fp4_bf16_nt(a, sfa, b, sfb, d, stream=None) -> None:
+    """d[M,N] (bf16) = a[M,K] (e4m3) . b^T, b packed e2m1 [N, K/2] bytes; scales as in
+    dg_gemm_fp8_fp8_bf16_nt."""
+    _fp8(a, "a")
+    _fp4(b, "b")
+    M, K = a.shape
+    N = b.shape[0]
+    if 2 * b.shape[1] != K:
+        raise ValueError("b must be [N, K/2] packed bytes")
+    _f32(sfa, "sfa", (K // BLOCK, get_tma_aligned_size(M, 4)))
+    _f32(sfb, "sfb", (-(-N // BLOCK), K // BLOCK))
+    _out(d, (M, N))
+    _check(lib.dg_gemm_fp8_fp4_bf16_nt(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K,
+                                       _stream(stream)), "dg_gemm_fp8_fp4_bf16_nt")
+
+
+def dg_m_grouped_gemm_fp8_fp4_bf16_nt_contiguous(a, sfa, b, sfb, d, m_indices, stream=None) -> None:
+    """Contiguous-layout grouped FP8 x FP4 GEMM: b packed e2m1 [G, N, K/2] bytes; everything
+    else as in dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous."""
+    _fp8(a, "a")
+    _fp4(b, "b")
+    M, K = a.shape
+    G, N, half_k = b.shape
+    if 2 * half_k != K:
+        raise ValueError("b must be [G, N, K/2] packed bytes")
+    _f32(sfa, "sfa", (K // BLOCK, get_tma_aligned_size(M, 4)))
+    _f32(sfb, "sfb", (G, -(-N // BLOCK), K // BLOCK))
+    _out(d, (M, N))
+    _i32(m_indices, "m_indices", (M,))
+    _check(lib.dg_m_grouped_gemm_fp8_fp4_bf16_nt_contiguous(
+        _ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), _ptr(m_indices), M, N, K, G,
+        _stream(stream)), "dg_m_grouped_gemm_fp8_fp4_bf16_nt_contiguous")
+
+
+def dg_m_grouped_gemm_fp8_fp4_bf16_nt_masked(a, sfa, b, sfb, d, masked_m, expected_m: int,
+                                             stream=None) -> None:
+    """Masked-layout grouped FP8 x FP4 GEMM: b packed e2m1 [G, N, K/2] bytes; everything else
+    as in dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked."""
+    _fp8(a, "a")
+    _fp4(b, "b")
+    G, M_max, K = a.shape
+    Gb, N, half_k = b.shape
+    if Gb != G or 2 * half_k != K:
+        raise ValueError("b must be [G, N, K/2] packed bytes with a's G")
+    _f32(sfa, "sfa", (G, K // BLOCK, get_tma_aligned_size(M_max, 4)))
+    _f32(sfb, "sfb", (G, -(-N // BLOCK), K // BLOCK))
+    _out(d, (G, M_max, N))
+    _i32(masked_m, "masked_m", (G,))
+    _check(lib.dg_m_grouped_gemm_fp8_fp4_bf16_nt_masked(
+        _ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), _ptr(masked_m), G, M_max, N, K,
+        int(expected_m), _stream(stream)), "dg_m_grouped_gemm_fp8_fp4_bf16_nt_masked")

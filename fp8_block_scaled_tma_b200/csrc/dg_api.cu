@@ -197,18 +197,23 @@ int stage_bytes_rt(int bn)
 
 
 
-// 4-D view [groups][K/128][rows][128 bytes] of a K-major uint8 operand: one box holds `kbs`
-// consecutive 128-wide K blocks of `box_rows` rows, laid out K block by K block in shared memory.
+// 4-D view [groups][K/128][rows][128 elements] of a K-major operand: one box holds `kbs`
+// consecutive 128-wide K blocks of `box_rows` rows, laid out K block by K block in shared memory,
+// 128 bytes per row and K block.  fp4: the operand is packed E2M1 (K/2 bytes per row), which
+// TMA expands into the padded layout tcgen05 kind::f8f6f4 reads (16 values in 8 bytes, then
+// 8 bytes of gap), so shared memory holds the same 128 bytes per row and K block as e4m3.
 int make_map_kblocks(CUtensorMap *map, void *base, uint64_t K, uint64_t rows, uint64_t groups,
-                     uint32_t box_rows, uint32_t kbs)
+                     uint32_t box_rows, uint32_t kbs, bool fp4 = false)
 {
+    const uint64_t row_bytes = fp4 ? K / 2 : K;
     cuuint64_t dims[4] = {128, rows, K / 128, groups};
-    cuuint64_t strides[3] = {K, 128, K * rows};
+    cuuint64_t strides[3] = {row_bytes, fp4 ? 64u : 128u, row_bytes * rows};
     cuuint32_t box[4] = {128, box_rows, kbs, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, base, dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = g_encode(map, fp4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                          4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
 }
 
@@ -439,6 +444,7 @@ struct LaunchArgs {
     int N, K, G;
     int expected_m;
     void *stream;
+    int b_fp4 = 0;  // B holds packed E2M1 (two per byte) instead of E4M3 codes
 };
 
 int launch_splitk(const LaunchArgs &args, int dev, DeviceInfo *info, int bn, int S,
@@ -489,8 +495,8 @@ int launch_splitk(const LaunchArgs &args, int dev, DeviceInfo *info, int bn, int
     CUtensorMap map_a, map_b;
     if (make_map_kblocks(&map_a, const_cast<void *>(args.a), K, M, 1, dg::kBlockM,
                          dg::kSplitKbPerStage) != DG_OK ||
-        make_map_kblocks(&map_b, const_cast<void *>(args.b), K, N, 1, bn, dg::kSplitKbPerStage) !=
-            DG_OK) {
+        make_map_kblocks(&map_b, const_cast<void *>(args.b), K, N, 1, bn, dg::kSplitKbPerStage,
+                         args.b_fp4 != 0) != DG_OK) {
         if (debug_enabled())
             std::fprintf(stderr, "[dg] cuTensorMapEncodeTiled failed (split-K)\n");
         return DG_ERR_CUDA;
@@ -514,6 +520,7 @@ int launch_splitk(const LaunchArgs &args, int dev, DeviceInfo *info, int bn, int
     p.err = info->err_ptr;
     p.timeout_ns = timeout;
     p.inject_stall = inject_stall_flag();
+    p.idesc_b = args.b_fp4 ? dg::ptx::kIdescBFormatE2M1 : 0u;
     p.num_tiles = m_tiles * n_tiles;
 
     cudaLaunchConfig_t cfg;
@@ -614,7 +621,7 @@ int launch_pair(const LaunchArgs &args, int dev, DeviceInfo *info, int sms, int 
         make_map_kblocks(&map_a, const_cast<void *>(args.a), K, M, a_groups, dg::kBlockM,
                          dg::kKbPerStage) != DG_OK ||
         make_map_kblocks(&map_b, const_cast<void *>(args.b), K, N, b_groups, bn / 2,
-                         dg::kKbPerStage) != DG_OK ||
+                         dg::kKbPerStage, args.b_fp4 != 0) != DG_OK ||
         // A scales [groups][K/128][align4(rows)]: one box = 128 rows x kKbPerStage K blocks
         make_map(&map_sfa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float *>(args.sfa), m4,
                  num_kb, a_groups, static_cast<uint64_t>(m4) * 4,
@@ -646,6 +653,7 @@ int launch_pair(const LaunchArgs &args, int dev, DeviceInfo *info, int sms, int 
     p.err = info->err_ptr;
     p.timeout_ns = timeout;
     p.inject_stall = inject_stall_flag();
+    p.idesc_b = args.b_fp4 ? dg::ptx::kIdescBFormatE2M1 : 0u;
     long long tiles = (args.layout == dg::kMasked)
                           ? static_cast<long long>(G) * pair_m_tiles * n_tiles
                           : static_cast<long long>(pair_m_tiles) * n_tiles;
@@ -841,9 +849,13 @@ int launch(const LaunchArgs &args)
         make_map(&map_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<void *>(args.a), K, a_rows,
                  a_groups, static_cast<uint64_t>(K), static_cast<uint64_t>(K) * a_rows, dg::kBlockK,
                  dg::kBlockM, CU_TENSOR_MAP_SWIZZLE_128B) != DG_OK ||
-        make_map(&map_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<void *>(args.b), K, N, b_groups,
-                 static_cast<uint64_t>(K), static_cast<uint64_t>(K) * N, dg::kBlockK, bn,
-                 CU_TENSOR_MAP_SWIZZLE_128B) != DG_OK) {
+        (args.b_fp4
+             ? make_map(&map_b, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, const_cast<void *>(args.b), K, N,
+                        b_groups, static_cast<uint64_t>(K) / 2, static_cast<uint64_t>(K) / 2 * N,
+                        dg::kBlockK, bn, CU_TENSOR_MAP_SWIZZLE_128B)
+             : make_map(&map_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<void *>(args.b), K, N,
+                        b_groups, static_cast<uint64_t>(K), static_cast<uint64_t>(K) * N, dg::kBlockK,
+                        bn, CU_TENSOR_MAP_SWIZZLE_128B)) != DG_OK) {
         if (debug_enabled())
             std::fprintf(stderr, "[dg] cuTensorMapEncodeTiled failed\n");
         return DG_ERR_CUDA;
@@ -870,6 +882,7 @@ int launch(const LaunchArgs &args)
     p.err = info->err_ptr;
     p.timeout_ns = timeout;
     p.inject_stall = inject_stall_flag();
+    p.idesc_b = args.b_fp4 ? dg::ptx::kIdescBFormatE2M1 : 0u;
     long long tiles;
     if (args.layout == dg::kMasked)
         tiles = static_cast<long long>(G) * m_tiles * n_tiles;  // upper bound; exact on device
@@ -1018,12 +1031,20 @@ int dg_quantize_fp8_1x128(const void *x, void *q, float *sfa, int M, int K, void
     return launch_quantize(x, q, sfa, M, K, stream);
 }
 
-int dg_gemm_fp8_fp8_bf16_nt(const void *a, const float *sfa, const void *b, const float *sfb,
-                            void *d, int M, int N, int K, void *workspace, size_t workspace_bytes,
-                            void *stream)
+}  // extern "C"
+
+namespace {
+
+// B of the FP8 x FP4 entries is packed E2M1; the tensor map for that layout wants a 32-byte
+// aligned base.
+bool b_aligned(const void *b, int b_fp4)
 {
-    (void)workspace;
-    (void)workspace_bytes;
+    return (reinterpret_cast<uintptr_t>(b) & (b_fp4 ? 31u : 15u)) == 0;
+}
+
+int gemm_dense(const void *a, const float *sfa, const void *b, const float *sfb, void *d, int M,
+               int N, int K, void *stream, int b_fp4)
+{
     if (M < 0)
         return DG_ERR_INVALID_ARG;
     if (M == 0)
@@ -1031,8 +1052,62 @@ int dg_gemm_fp8_fp8_bf16_nt(const void *a, const float *sfa, const void *b, cons
     int st = check_common(a, sfa, b, sfb, d, N, K);
     if (st != DG_OK)
         return st;
-    LaunchArgs la{dg::kDense, a, sfa, b, sfb, d, nullptr, nullptr, M, N, K, 1, 0, stream};
+    if (!b_aligned(b, b_fp4))
+        return DG_ERR_INVALID_ARG;
+    LaunchArgs la{dg::kDense, a, sfa, b, sfb, d, nullptr, nullptr, M, N, K, 1, 0, stream, b_fp4};
     return launch(la);
+}
+
+int gemm_contiguous(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
+                    const int *m_indices, int M_total, int N, int K, int G, void *stream, int b_fp4)
+{
+    if (M_total < 0 || M_total % dg::kBlockM != 0 || G <= 0)
+        return DG_ERR_INVALID_ARG;
+    if (M_total == 0)
+        return (N > 0 && N % 8 == 0 && K > 0 && K % dg::kBlockK == 0) ? DG_OK : DG_ERR_INVALID_ARG;
+    int st = check_common(a, sfa, b, sfb, d, N, K);
+    if (st != DG_OK)
+        return st;
+    if (!b_aligned(b, b_fp4))
+        return DG_ERR_INVALID_ARG;
+    if (!m_indices || (reinterpret_cast<uintptr_t>(m_indices) & 3u))
+        return DG_ERR_INVALID_ARG;
+    LaunchArgs la{dg::kContiguous, a, sfa, b, sfb, d, m_indices, nullptr, M_total, N, K, G, 0,
+                  stream, b_fp4};
+    return launch(la);
+}
+
+int gemm_masked(const void *a, const float *sfa, const void *b, const float *sfb, void *d,
+                const int *masked_m, int G, int M_max, int N, int K, int expected_m, void *stream,
+                int b_fp4)
+{
+    if (G <= 0 || G > dg::kMaxMaskedGroups || M_max < 0 || expected_m < 0)
+        return DG_ERR_INVALID_ARG;
+    if (M_max == 0)
+        return (N > 0 && N % 8 == 0 && K > 0 && K % dg::kBlockK == 0) ? DG_OK : DG_ERR_INVALID_ARG;
+    int st = check_common(a, sfa, b, sfb, d, N, K);
+    if (st != DG_OK)
+        return st;
+    if (!b_aligned(b, b_fp4))
+        return DG_ERR_INVALID_ARG;
+    if (!masked_m || (reinterpret_cast<uintptr_t>(masked_m) & 3u))
+        return DG_ERR_INVALID_ARG;
+    LaunchArgs la{dg::kMasked, a, sfa, b, sfb, d, nullptr, masked_m, M_max, N, K, G, expected_m,
+                  stream, b_fp4};
+    return launch(la);
+}
+
+}  // namespace
+
+extern "C" {
+
+int dg_gemm_fp8_fp8_bf16_nt(const void *a, const float *sfa, const void *b, const float *sfb,
+                            void *d, int M, int N, int K, void *workspace, size_t workspace_bytes,
+                            void *stream)
+{
+    (void)workspace;
+    (void)workspace_bytes;
+    return gemm_dense(a, sfa, b, sfb, d, M, N, K, stream, 0);
 }
 
 int dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(const void *a, const float *sfa, const void *b,
@@ -1042,18 +1117,7 @@ int dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(const void *a, const float *sfa
 {
     (void)workspace;
     (void)workspace_bytes;
-    if (M_total < 0 || M_total % dg::kBlockM != 0 || G <= 0)
-        return DG_ERR_INVALID_ARG;
-    if (M_total == 0)
-        return (N > 0 && N % 8 == 0 && K > 0 && K % dg::kBlockK == 0) ? DG_OK : DG_ERR_INVALID_ARG;
-    int st = check_common(a, sfa, b, sfb, d, N, K);
-    if (st != DG_OK)
-        return st;
-    if (!m_indices || (reinterpret_cast<uintptr_t>(m_indices) & 3u))
-        return DG_ERR_INVALID_ARG;
-    LaunchArgs la{dg::kContiguous, a, sfa, b, sfb, d, m_indices, nullptr, M_total, N, K, G, 0,
-                  stream};
-    return launch(la);
+    return gemm_contiguous(a, sfa, b, sfb, d, m_indices, M_total, N, K, G, stream, 0);
 }
 
 int dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked(const void *a, const float *sfa, const void *b,
@@ -1063,18 +1127,27 @@ int dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked(const void *a, const float *sfa, co
 {
     (void)workspace;
     (void)workspace_bytes;
-    if (G <= 0 || G > dg::kMaxMaskedGroups || M_max < 0 || expected_m < 0)
-        return DG_ERR_INVALID_ARG;
-    if (M_max == 0)
-        return (N > 0 && N % 8 == 0 && K > 0 && K % dg::kBlockK == 0) ? DG_OK : DG_ERR_INVALID_ARG;
-    int st = check_common(a, sfa, b, sfb, d, N, K);
-    if (st != DG_OK)
-        return st;
-    if (!masked_m || (reinterpret_cast<uintptr_t>(masked_m) & 3u))
-        return DG_ERR_INVALID_ARG;
-    LaunchArgs la{dg::kMasked, a, sfa, b, sfb, d, nullptr, masked_m, M_max, N, K, G, expected_m,
-                  stream};
-    return launch(la);
+    return gemm_masked(a, sfa, b, sfb, d, masked_m, G, M_max, N, K, expected_m, stream, 0);
+}
+
+int dg_gemm_fp8_fp4_bf16_nt(const void *a, const float *sfa, const void *b, const float *sfb,
+                            void *d, int M, int N, int K, void *stream)
+{
+    return gemm_dense(a, sfa, b, sfb, d, M, N, K, stream, 1);
+}
+
+int dg_m_grouped_gemm_fp8_fp4_bf16_nt_contiguous(const void *a, const float *sfa, const void *b,
+                                                 const float *sfb, void *d, const int *m_indices,
+                                                 int M_total, int N, int K, int G, void *stream)
+{
+    return gemm_contiguous(a, sfa, b, sfb, d, m_indices, M_total, N, K, G, stream, 1);
+}
+
+int dg_m_grouped_gemm_fp8_fp4_bf16_nt_masked(const void *a, const float *sfa, const void *b,
+                                             const float *sfb, void *d, const int *masked_m, int G,
+                                             int M_max, int N, int K, int expected_m, void *stream)
+{
+    return gemm_masked(a, sfa, b, sfb, d, masked_m, G, M_max, N, K, expected_m, stream, 1);
 }
 
 int dg_set_num_sms(int n)

@@ -70,6 +70,8 @@ struct Params {
     int *err;
     unsigned long long timeout_ns;
     int inject_stall;   // test hook: the MMA issuer first waits on a barrier nothing signals
+    uint32_t idesc_b;   // B-format bits of the MMA instruction descriptor: 0 e4m3, or e2m1
+                        // (FP4 B, staged by TMA in the padded 8-bit layout of kind::f8f6f4)
 };
 
 template <int BN>
@@ -84,6 +86,9 @@ struct Cfg {
     static constexpr int kBBytes = BN * kBlockK;
     static constexpr int kStageBytes = kABytes + kBBytes;     // multiple of 1024
     static constexpr uint32_t kTxBytes = kABytes + kBBytes;
+    // TMA counts a packed E2M1 operand at 4 bits per element, though it lands in shared memory
+    // at 8 bits per element (16 values, then 8 bytes of gap)
+    static constexpr uint32_t kTxBytesFp4B = kABytes + kBBytes / 2;
     static constexpr uint32_t kIdesc = ptx::idesc_e4m3_f32(kBlockM, BN);
 };
 
@@ -601,7 +606,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     }
                     if (ptx::elect_one()) {
                         const uint32_t fb = bar_full + 8 * s;
-                        ptx::mbar_arrive_expect_tx(fb, C::kTxBytes);
+                        ptx::mbar_arrive_expect_tx(fb, p.idesc_b ? C::kTxBytesFp4B : C::kTxBytes);
                         ptx::tma_load_3d(stage_a(s), &tmap_a, fb, kb * kBlockK, ti.m0, ti.a_z);
                         ptx::tma_load_3d(stage_b(s), &tmap_b, fb, kb * kBlockK, n0, ti.g);
                     }
@@ -656,7 +661,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 #pragma unroll
                         for (int k = 0; k < kBlockK / kUmmaK; ++k) {
                             // advance the start address by 32 bytes (2 x 16 B) per K step
-                            ptx::mma_f8f6f4(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::kIdesc,
+                            ptx::mma_f8f6f4(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::kIdesc | p.idesc_b,
                                             k > 0 ? 1u : 0u);
                         }
                         ptx::mma_commit(bar_empty + 8 * s);

@@ -37,6 +37,7 @@ struct PairCfg {
     static constexpr int kBBytes = kKbPerStage * kBKbBytes;
     static constexpr int kStageBytes = kABytes + kBBytes;          // multiple of 1024
     static constexpr uint32_t kTxBytesPerCta = kABytes + kBBytes;
+    static constexpr uint32_t kTxBytesPerCtaFp4B = kABytes + kBBytes / 2;  // packed E2M1 B
     static constexpr uint32_t kIdesc = ptx::idesc_e4m3_f32(2 * kBlockM, BN);
     static constexpr int kSfaSlotBytes = kKbPerStage * kBlockM * 4;  // A scales of one stage
 };
@@ -238,7 +239,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     }
                     if (ptx::elect_one()) {
                         const uint32_t fb = full0 + 8 * s;
-                        ptx::mbar_arrive_expect_tx_cluster(fb, C::kTxBytesPerCta);
+                        ptx::mbar_arrive_expect_tx_cluster(fb, p.idesc_b ? C::kTxBytesPerCtaFp4B : C::kTxBytesPerCta);
                         ptx::tma_load_4d_pair(stage_a(s), &tmap_a, fb, 0, a_row, kb0, ti.a_z);
                         ptx::tma_load_4d_pair(stage_b(s), &tmap_b, fb, 0, b_row, kb0, ti.g);
                     }
@@ -307,7 +308,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                             const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
 #pragma unroll
                             for (int k = 0; k < kBlockK / kUmmaK; ++k)
-                                ptx::mma_f8f6f4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::kIdesc,
+                                ptx::mma_f8f6f4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::kIdesc | p.idesc_b,
                                                      k > 0 ? 1u : 0u);
                             ptx::mma_commit_pair_multicast(bar_tfull + 8 * buf, 0x3);
                         }

@@ -195,6 +195,10 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int m, int n)
            (static_cast<uint32_t>(m >> 4) << 24);
 }
 
+// B-format field (bits 10-12) of a kind::f8f6f4 instruction descriptor for E2M1 (FP4) B,
+// OR'ed into idesc_e4m3_f32: A stays e4m3.
+constexpr uint32_t kIdescBFormatE2M1 = 5u << 10;
+
 // ---- tcgen05: TMEM -> registers ------------------------------------------------------------
 
 // 32 lanes x 32 bits, 16 consecutive columns per thread.

@@ -32,6 +32,7 @@ struct SplitCfg {
     static constexpr int kABytes = kSplitKbPerStage * kAKbBytes;
     static constexpr int kStageBytes = kSplitKbPerStage * (kAKbBytes + kBKbBytes);
     static constexpr uint32_t kTxBytes = kStageBytes;
+    static constexpr uint32_t kTxBytesFp4B = kSplitKbPerStage * (kAKbBytes + kBKbBytes / 2);  // packed E2M1 B
     static constexpr uint32_t kIdesc = ptx::idesc_e4m3_f32(kBlockM, BN);
     static constexpr int kPartLd = BN + 4;  // fp32 row stride of the partial tile (bank spread)
     static constexpr int kPartBytes = kBlockM * kPartLd * 4;
@@ -129,7 +130,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         if (ptx::elect_one()) {
             for (int i = 0; i < pre; ++i) {
                 const uint32_t fb = bar_full + 8 * i;
-                ptx::mbar_arrive_expect_tx(fb, C::kTxBytes);
+                ptx::mbar_arrive_expect_tx(fb, p.idesc_b ? C::kTxBytesFp4B : C::kTxBytes);
                 ptx::tma_load_4d(stage_a(i), &tmap_a, fb, 0, m0, kb_begin + i * KS, 0);
                 ptx::tma_load_4d(stage_b(i), &tmap_b, fb, 0, n0, kb_begin + i * KS, 0);
             }
@@ -158,7 +159,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                     break;
                 if (ptx::elect_one()) {
                     const uint32_t fb = bar_full + 8 * s;
-                    ptx::mbar_arrive_expect_tx(fb, C::kTxBytes);
+                    ptx::mbar_arrive_expect_tx(fb, p.idesc_b ? C::kTxBytesFp4B : C::kTxBytes);
                     ptx::tma_load_4d(stage_a(s), &tmap_a, fb, 0, m0, kb0, 0);
                     ptx::tma_load_4d(stage_b(s), &tmap_b, fb, 0, n0, kb0, 0);
                 }
@@ -204,7 +205,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
 #pragma unroll
                         for (int k = 0; k < kBlockK / kUmmaK; ++k)
-                            ptx::mma_f8f6f4(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::kIdesc,
+                            ptx::mma_f8f6f4(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::kIdesc | p.idesc_b,
                                             k > 0 ? 1u : 0u);
                         ptx::mma_commit(bar_tfull + 8 * buf);
                     }

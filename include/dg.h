@@ -94,6 +94,30 @@ int dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked(const void *a, const float *sfa, co
                                              void *workspace, size_t workspace_bytes,
                                              void *stream);
 
+/* FP8 x FP4 variants: the mixed-precision "FP8 x FP4" matrix multiplication that the DeepGEMM
+ * update news item ("Perpustakaan operator GPU sumber terbuka DeepSeek DeepGEMM memperbarui
+ * versi besar ...") lists among the additions.  The item fixes neither the FP4 format, its
+ * layout nor its scales; these calls take the plainest reading:
+ *   - b holds OCP FP4 E2M1 values (sign, 2 exponent bits with bias 1, 1 mantissa bit; values
+ *     +-{0, 0.5, 1, 1.5, 2, 3, 4, 6}), packed two per byte along K: element k of a row is the
+ *     low nibble of byte k/2 when k is even, the high nibble when k is odd.  A row of b is
+ *     K/2 bytes; groups follow each other ([G][N][K/2] for the grouped calls).
+ *   - sfb is unchanged: one fp32 scale per 128 x 128 block of b, [G][N/128][K/128].
+ *   - a, sfa, d, m_indices, masked_m and every other rule are those of the FP8 x FP8 call of
+ *     the same name, and the result is the same formula with b's E2M1 values in place of e4m3.
+ * The tensor cores take e4m3 x e2m1 directly; nothing is converted in memory.  b must be 32-byte
+ * aligned (DG_ERR_INVALID_ARG otherwise).  No workspace is used. */
+int dg_gemm_fp8_fp4_bf16_nt(const void *a, const float *sfa, const void *b, const float *sfb,
+                            void *d, int M, int N, int K, void *stream);
+
+int dg_m_grouped_gemm_fp8_fp4_bf16_nt_contiguous(const void *a, const float *sfa, const void *b,
+                                                 const float *sfb, void *d, const int *m_indices,
+                                                 int M_total, int N, int K, int G, void *stream);
+
+int dg_m_grouped_gemm_fp8_fp4_bf16_nt_masked(const void *a, const float *sfa, const void *b,
+                                             const float *sfb, void *d, const int *masked_m, int G,
+                                             int M_max, int N, int K, int expected_m, void *stream);
+
 /* Per-token FP8 quantisation of activations: the step that produces the GEMMs' A operand and
  * its scales (the fine-grained 1 x 128 activation scaling of "深入了解DeepGEMM", written in the
  * TMA-aligned scale layout that the utility functions of "如何使用" serve).  For each row m and

@@ -119,8 +119,9 @@ uint8_t orc_e4m3_encode(float v)
     return sign | (uint8_t)(code > 0x7E ? 0x7E : code);
 }
 
-/* OCP 4-bit floating point E2M1 (the FP4 of FP8 x FP4 GEMMs, the later DeepGEMM release, page
- * 2): bit 3 the sign, bits 2..1 the exponent (bias 1), bit 0 the mantissa; exponent 0 is
+/* OCP 4-bit floating point E2M1 (the FP4 of the FP8 x FP4 GEMM that the DeepGEMM update news
+ * item, "Perpustakaan operator GPU sumber terbuka DeepSeek DeepGEMM memperbarui versi besar",
+ * lists among the additions): bit 3 the sign, bits 2..1 the exponent (bias 1), bit 0 the mantissa; exponent 0 is
  * subnormal (m / 2).  Values +-{0, 0.5, 1, 1.5, 2, 3, 4, 6}; no infinities or NaN. */
 double orc_e2m1_decode(uint8_t nibble)
 {

@@ -110,6 +110,43 @@ def run_masked(dg, case, a=None, sa=None) -> torch.Tensor:
     return d
 
 
+def run_dense_fp4(dg, case, d=None) -> torch.Tensor:
+    """case.b holds packed E2M1 bytes [N, K/2]."""
+    a = to_dev_u8(case.a)
+    b = to_dev_u8(case.b)
+    sfa = dg.sfa_mn_major(to_dev_f32(case.sa))
+    sfb = to_dev_f32(case.sb)
+    if d is None:
+        d = sentinel_out((case.M, case.N))
+    dg.dg_gemm_fp8_fp4_bf16_nt(a, sfa, b, sfb, d)
+    torch.cuda.synchronize()
+    return d
+
+
+def run_contiguous_fp4(dg, case) -> torch.Tensor:
+    a = to_dev_u8(case.a)
+    sfa = dg.sfa_mn_major(to_dev_f32(case.sa))
+    b = to_dev_u8(case.b)
+    sfb = to_dev_f32(case.sb)
+    mi = torch.from_numpy(case.m_indices).cuda()
+    d = sentinel_out((case.M_total, case.N))
+    dg.dg_m_grouped_gemm_fp8_fp4_bf16_nt_contiguous(a, sfa, b, sfb, d, mi)
+    torch.cuda.synchronize()
+    return d
+
+
+def run_masked_fp4(dg, case) -> torch.Tensor:
+    a = to_dev_u8(case.a)
+    sfa = dg.sfa_mn_major(to_dev_f32(case.sa))
+    b = to_dev_u8(case.b)
+    sfb = to_dev_f32(case.sb)
+    mm = torch.from_numpy(case.masked_m).cuda()
+    d = sentinel_out((case.G, case.M_max, case.N))
+    dg.dg_m_grouped_gemm_fp8_fp4_bf16_nt_masked(a, sfa, b, sfb, d, mm, case.expected_m)
+    torch.cuda.synchronize()
+    return d
+
+
 def sample_rows(M: int, n: int, seed: int) -> np.ndarray:
     """Rows at tile boundaries (first/last rows of the first, second and last 128-row tiles)
     plus n seeded random rows."""

@@ -32,7 +32,9 @@ def test_header_declares_the_api():
     names = declared_functions()
     for n in ["dg_gemm_fp8_fp8_bf16_nt", "dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous",
               "dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked", "dg_set_num_sms", "dg_get_num_sms",
-              "dg_get_tma_aligned_size"]:
+              "dg_get_tma_aligned_size", "dg_gemm_fp8_fp4_bf16_nt",
+              "dg_m_grouped_gemm_fp8_fp4_bf16_nt_contiguous",
+              "dg_m_grouped_gemm_fp8_fp4_bf16_nt_masked"]:
         assert n in names
 
 
@@ -126,6 +128,28 @@ def test_grouped_reject_bad_arguments(dg):
                                                       256, 256, -1, None, 0, None) == -1
     assert L.dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked(FAKE, FAKE, FAKE, FAKE, FAKE, None, 2, 256,
                                                       256, 256, 128, None, 0, None) == -1
+
+
+def test_fp4_entries_reject_bad_arguments(dg):
+    L = dg.lib
+    # packed E2M1 B must be 32-byte aligned (16 is enough for e4m3 B)
+    assert L.dg_gemm_fp8_fp4_bf16_nt(FAKE, FAKE, FAKE + 16, FAKE, FAKE, 128, 256, 256, None) == -1
+    assert L.dg_gemm_fp8_fp4_bf16_nt(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 256, 200, None) == -1
+    assert L.dg_gemm_fp8_fp4_bf16_nt(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 256, 256, None) == 0
+    assert L.dg_m_grouped_gemm_fp8_fp4_bf16_nt_contiguous(FAKE, FAKE, FAKE + 16, FAKE, FAKE, FAKE,
+                                                          128, 256, 256, 2, None) == -1
+    assert L.dg_m_grouped_gemm_fp8_fp4_bf16_nt_contiguous(FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                                                          128, 256, 256, 2, None) == -1
+    assert L.dg_m_grouped_gemm_fp8_fp4_bf16_nt_masked(FAKE, FAKE, FAKE + 16, FAKE, FAKE, FAKE, 2,
+                                                      128, 256, 256, 64, None) == -1
+    assert L.dg_m_grouped_gemm_fp8_fp4_bf16_nt_masked(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0,
+                                                      128, 256, 256, 64, None) == -1
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_fp4_valid_call_without_device_is_unsupported(dg):
+    r = dg.lib.dg_gemm_fp8_fp4_bf16_nt(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 256, 256, None)
+    assert r == dg.DG_ERR_UNSUPPORTED
 
 
 def test_empty_problems_are_noops(dg):

@@ -1,5 +1,5 @@
 """Pins of the oracle's FP4 (E2M1) operand path of the FP8 x FP4 GEMM (the mixed-precision
-variant of the later DeepGEMM release, page 2): the E2M1 value table that the OCP format
+variant that the DeepGEMM update news item lists): the E2M1 value table that the OCP format
 definition fixes, the exactness of its expansion into E4M3 codes, the nibble order of the packed
 layout, and a small FP8 x FP4 GEMM checked in exact rational arithmetic."""
 from __future__ import annotations

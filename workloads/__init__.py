@@ -177,6 +177,20 @@ def masked(G: int, M_max: int, N: int, K: int, seed: int, expected_m: int = 128,
     return Masked(G, M_max, N, K, expected_m, masked_m, a, sa, b, sb)
 
 
+def with_fp4_b(case, seed: int, b_std: float = 0.02):
+    """A copy of a Dense / Contiguous / Masked case whose B is an FP4 (E2M1) operand: packed
+    bytes [.., N, K/2] drawn uniformly (so every one of the 16 codes, -0 included, occurs in
+    both nibble positions; element 2j of a row is the low nibble of byte j) and fresh 128x128
+    block scales uniform in [0.5, 1.5] * b_std * 4/6 (the size an absmax/6 scaling of
+    N(0, b_std^2) weights gives).  A, its scales and the layout fields are kept."""
+    import dataclasses
+    g = _gen(seed)
+    b_shape = case.b.shape[:-1] + (case.b.shape[-1] // 2,)
+    b = torch.randint(0, 256, b_shape, generator=g, dtype=torch.int32).to(torch.uint8).numpy()
+    sb = ((torch.rand(case.sb.shape, generator=g) + 0.5) * (b_std * 4.0 / 6.0)).float().numpy()
+    return dataclasses.replace(case, b=b, sb=sb)
+
+
 # ---- the named workloads ----------------------------------------------------------------
 
 SMALL_DENSE = dict(M=128, N=256, K=512)
