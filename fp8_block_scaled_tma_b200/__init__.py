@@ -205,7 +205,8 @@ FAMILY_AUTO, FAMILY_ONE_CTA, FAMILY_PAIR, FAMILY_SPLIT_K = 0, 1, 2, 3
 
 def set_kernel_family(family: int) -> int:
     """0 automatic, 1 one-CTA kernels, 2 CTA-pair kernels where the layout allows, 3 split-K
-    cluster kernel for dense calls.  Returns the previous value."""
+    cluster kernel for dense calls, 4 swapped-operand kernel for dense calls with M <= 128.
+    Returns the previous value."""
     r = lib.dg_set_kernel_family(int(family))
     if r < 0:
         raise DGError(r, "dg_set_kernel_family")

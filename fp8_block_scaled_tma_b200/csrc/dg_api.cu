@@ -15,6 +15,7 @@
 #include "dg_pair_kernel.cuh"
 #include "dg_quant_kernel.cuh"
 #include "dg_splitk_kernel.cuh"
+#include "dg_swap_kernel.cuh"
 
 namespace {
 
@@ -43,7 +44,10 @@ struct KernelSmem {
 KernelSmem g_smem[kMaxDevices][3][8];       // 1-CTA kernels, per device / layout / BN
 KernelSmem g_smem_pair[kMaxDevices][3][8];  // CTA-pair kernels
 KernelSmem g_smem_split[kMaxDevices][8];    // split-K kernels, per BN
-int g_family = 0;  // 0 auto, 1 one-CTA kernels, 2 CTA pairs where possible, 3 split-K (dense)
+KernelSmem g_smem_swap[kMaxDevices][6];     // swapped-operand kernels, per (TN, R)
+// 0 auto, 1 one-CTA kernels, 2 CTA pairs where possible, 3 split-K (dense), 4 swapped operands
+// (dense, M <= 128)
+int g_family = 0;
 int g_num_sms_cap = 0;
 unsigned long long g_timeout_ns = kDefaultTimeoutNs;
 int g_override_bn = 0;
@@ -53,7 +57,7 @@ int g_inject_stall = 0;
 int g_pdl = 1;  // launch with programmatic stream serialisation (dg_set_pdl)
 // clusters of each size (index = cluster size, 1..8) that can be resident at once, per device
 // and kernel family; 0 = not queried yet
-int g_max_clusters[kMaxDevices][3][9];
+int g_max_clusters[kMaxDevices][9][9];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 struct LastLaunch {
@@ -702,6 +706,218 @@ int launch_pair(const LaunchArgs &args, int dev, DeviceInfo *info, int sms, int 
     return DG_OK;
 }
 
+// ---- swapped-operand kernel (dense, M <= 128) ------------------------------------------------
+
+int swap_index(int tn, int R)
+{
+    const int t = tn == 32 ? 0 : tn == 64 ? 1 : tn == 128 ? 2 : -1;
+    return (t < 0 || (R != 1 && R != 2)) ? -1 : t * 2 + (R - 1);
+}
+
+template <int TN, int R>
+void *swap_kernel_ptr()
+{
+    return reinterpret_cast<void *>(&dg::dg_gemm_swap_kernel<TN, R>);
+}
+
+void *pick_swap_kernel(int tn, int R)
+{
+    switch (swap_index(tn, R)) {
+    case 0: return swap_kernel_ptr<32, 1>();
+    case 1: return swap_kernel_ptr<32, 2>();
+    case 2: return swap_kernel_ptr<64, 1>();
+    case 3: return swap_kernel_ptr<64, 2>();
+    case 4: return swap_kernel_ptr<128, 1>();
+    case 5: return swap_kernel_ptr<128, 2>();
+    default: return nullptr;
+    }
+}
+
+int swap_token_tile(int M)
+{
+    return M <= 32 ? 32 : M <= 64 ? 64 : 128;
+}
+
+int swap_stage_bytes(int tn, int R)
+{
+    return dg::kSwapKbPerStage * (R * dg::kBlockM * dg::kBlockK + tn * dg::kBlockK);
+}
+
+int swap_scale_bytes(int tn, int R, int kb_box)
+{
+    return kb_box * tn * 4 * (R == 1 ? 1 : 3);
+}
+
+// Choice of R (128-row blocks of B per tile) and S (K splits = cluster size) for the
+// swapped-operand kernel.  Time model: the problem cannot beat HBM, a CTA cannot pull more
+// than ~80 GB/s through its TMA pipeline, and with S > 1 the cluster barriers and the
+// reduction through distributed shared memory cost ~0.26 us per split plus ~0.14 ns per partial
+// element (the split-K kernel's fitted constants).  Returns false if nothing fits in one wave.
+template <class Capacity>
+bool choose_swap(int M, int N, int K, bool fp4, int sms, int dyn_cap, int r_fixed, int s_fixed,
+                 Capacity capacity, int &r_out, int &s_out)
+{
+    const int num_kb = K / dg::kBlockK;
+    const int nblocks = (N + dg::kBlockM - 1) / dg::kBlockM;
+    const int tn = swap_token_tile(M);
+    const double b_bytes = static_cast<double>(N) * K * (fp4 ? 0.5 : 1.0);
+    const double t_hbm = (b_bytes + static_cast<double>(M) * K) / 6500.0;  // ns
+    double best = 1e300;
+    bool found = false;
+    for (int R = 1; R <= 2; ++R) {
+        if (r_fixed != 0 && R != r_fixed)
+            continue;
+        const long long tiles = (nblocks + R - 1) / R;
+        for (int S = 1; S <= dg::kMaxSplits; ++S) {
+            if (s_fixed != 0 && S != s_fixed)
+                continue;
+            if (S > num_kb)
+                continue;
+            const int kb_box = (num_kb + S - 1) / S;
+            if (kb_box > 256 || swap_scale_bytes(tn, R, kb_box) > dg::kSwapMaxScaleBytes)
+                continue;
+            // at least two operand stages, which also hold the fp32 partial after the K loop
+            const int sbytes = swap_stage_bytes(tn, R);
+            const int stages = std::min(dg::kMaxStages, (dyn_cap - 1024 - swap_scale_bytes(tn, R, kb_box)) / sbytes);
+            if (stages < 2 || stages * sbytes < tn * R * dg::kBlockM * 4)
+                continue;
+            if (tiles * S > sms || tiles > capacity(tn, R, S))
+                continue;
+            const double kb_bytes = R * dg::kBlockM * dg::kBlockK * (fp4 ? 0.5 : 1.0) +
+                                    static_cast<double>(tn) * dg::kBlockK;
+            const double t_cta = kb_box * kb_bytes / 80.0;
+            const double t_red = S > 1 ? 263.0 * S + 0.139 * std::min(M, tn) * R * dg::kBlockM : 0.0;
+            const double t = std::max(t_hbm, t_cta) + t_red;
+            if (t < best - 1e-9) {
+                best = t;
+                r_out = R;
+                s_out = S;
+                found = true;
+            }
+        }
+    }
+    return found;
+}
+
+int launch_swap(const LaunchArgs &args, int dev, DeviceInfo *info, int R, int S,
+                int stages_override, unsigned long long timeout)
+{
+    const int M = args.M, N = args.N, K = args.K;
+    const int num_kb = K / dg::kBlockK;
+    const int num_nb = (N + dg::kBlockK - 1) / dg::kBlockK;
+    const int tn = swap_token_tile(M);
+    const int idx = swap_index(tn, R);
+    void *fn = pick_swap_kernel(tn, R);
+    if (fn == nullptr || M > 128 || S < 1 || S > dg::kMaxSplits || S > num_kb)
+        return DG_ERR_INVALID_ARG;
+    const int n_tiles = (N + R * dg::kBlockM - 1) / (R * dg::kBlockM);
+    const int kb_box = (num_kb + S - 1) / S;
+    const int sbytes = swap_stage_bytes(tn, R);
+    const int scale_bytes = swap_scale_bytes(tn, R, kb_box);
+    const int part_bytes = tn * R * dg::kBlockM * 4;
+    if (kb_box > 256 || scale_bytes > dg::kSwapMaxScaleBytes)
+        return DG_ERR_UNSUPPORTED;
+    int stages = 0, dyn_smem = 0;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        KernelSmem &ks = g_smem_swap[dev][idx];
+        if (ks.static_bytes < 0) {
+            cudaFuncAttributes fa;
+            cudaError_t e = cudaFuncGetAttributes(&fa, fn);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                return DG_ERR_CUDA;
+            }
+            ks.static_bytes = static_cast<int>(fa.sharedSizeBytes);
+        }
+        const int dyn_cap = info->smem_optin - ks.static_bytes;
+        stages = std::min(dg::kMaxStages, (dyn_cap - 1024 - scale_bytes) / sbytes);
+        if (stages_override > 0)
+            stages = std::min(stages, stages_override);
+        // the operand stages are reused for the fp32 partial after the K loop
+        if (stages < 2 || stages * sbytes < part_bytes)
+            return DG_ERR_UNSUPPORTED;
+        dyn_smem = stages * sbytes + scale_bytes + 1024;
+        dyn_smem = std::min(std::max(dyn_smem, kMinDynSmem), dyn_cap);
+        if (ks.limit_set < dyn_smem) {
+            cudaError_t e =
+                cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                return DG_ERR_CUDA;
+            }
+            ks.limit_set = dyn_smem;
+        }
+    }
+    const int sfa_ld = align4(M);
+    CUtensorMap map_a, map_b, map_sa;
+    if (make_map_kblocks(&map_a, const_cast<void *>(args.a), K, M, 1, tn, dg::kSwapKbPerStage) != DG_OK ||
+        make_map_kblocks(&map_b, const_cast<void *>(args.b), K, N, 1, R * dg::kBlockM,
+                         dg::kSwapKbPerStage, args.b_fp4 != 0) != DG_OK ||
+        make_map(&map_sa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float *>(args.sfa), sfa_ld,
+                 num_kb, 1, static_cast<uint64_t>(sfa_ld) * 4, static_cast<uint64_t>(sfa_ld) * 4 * num_kb,
+                 tn, kb_box, CU_TENSOR_MAP_SWIZZLE_NONE) != DG_OK) {
+        if (debug_enabled())
+            std::fprintf(stderr, "[dg] cuTensorMapEncodeTiled failed (swapped operands)\n");
+        return DG_ERR_CUDA;
+    }
+    Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.G = 1;
+    p.num_kb = num_kb;
+    p.num_nb = num_nb;
+    p.m_tiles = kb_box;
+    p.n_tiles = n_tiles;
+    p.stages = stages;
+    p.raster_m = S;
+    p.sfa = args.sfa;
+    p.sfa_ld = sfa_ld;
+    p.sfb = args.sfb;
+    p.d = static_cast<__nv_bfloat16 *>(args.d);
+    p.err = info->err_ptr;
+    p.timeout_ns = timeout;
+    p.inject_stall = inject_stall_flag();
+    p.idesc_b = args.b_fp4 ? dg::ptx::kIdescBFormatE2M1 : 0u;
+    p.num_tiles = n_tiles;
+
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(n_tiles * S, 1, 1);
+    cfg.blockDim = dim3(dg::kNumThreads, 1, 1);
+    cfg.dynamicSmemBytes = dyn_smem;
+    cfg.stream = static_cast<cudaStream_t>(args.stream);
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = add_pdl_attr(attr, 1);
+    void *kargs[] = {&map_a, &map_b, &map_sa, &p};
+    cudaError_t e = cudaLaunchKernelExC(&cfg, fn, kargs);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        if (debug_enabled())
+            std::fprintf(stderr, "[dg] swapped-operand launch failed: %s\n", cudaGetErrorString(e));
+        return DG_ERR_CUDA;
+    }
+    t_last.valid = true;
+    t_last.block_n = R * dg::kBlockM;
+    t_last.stages = stages;
+    t_last.grid = n_tiles * S;
+    t_last.tiles = n_tiles;
+    t_last.pair = 0;
+    t_last.splits = S;
+    t_last.family = 4;
+    if (debug_enabled())
+        std::fprintf(stderr, "[dg] swap M=%d N=%d K=%d TN=%d R=%d S=%d stages=%d grid=%d smem=%d\n", M,
+                     N, K, tn, R, S, stages, n_tiles * S, dyn_smem);
+    return DG_OK;
+}
+
 int launch(const LaunchArgs &args)
 {
     int dev = 0;
@@ -733,6 +949,43 @@ int launch(const LaunchArgs &args)
         timeout = g_timeout_ns;
         pair_mode = g_family;
     }
+    // Swapped operands for dense problems with few rows (decode-sized token counts): B rows on
+    // the MMA's 128-lane side, the tokens on its N side.  Family 4 forces it for M <= 128.  Auto
+    // mode takes it for M <= 64 with one 128-row block of B per tile, where it measured ahead of
+    // split-K on B200 (1-2 us on the 2112 / 4096 / 7168-wide decode shapes); with 65-128 tokens,
+    // or when the tiles need two row blocks to fit in one wave, split-K and the one-CTA kernel
+    // were level or faster.  (In auto mode a block_n override keeps the families it names.)
+    const bool swap_auto = pair_mode == 0 && bn == 0 && M <= 64;
+    if (args.layout == dg::kDense && M <= 128 && (pair_mode == 4 || swap_auto)) {
+        int splits_override;
+        {
+            std::lock_guard<std::mutex> lock(g_mutex);
+            splits_override = g_override_splits;
+        }
+        const int r_fixed = bn == 128 ? 1 : bn == 256 ? 2 : (pair_mode == 0 ? 1 : 0);
+        auto capacity = [&](int ctn, int cR, int cs) -> long long {
+            void *fn = pick_swap_kernel(ctn, cR);
+            const int smem = std::max(std::min(2 * swap_stage_bytes(ctn, cR) + 16 * 1024, 200 * 1024),
+                                      kMinDynSmem);
+            int n = max_active_clusters(fn, cs, smem, dev, 3 + swap_index(ctn, cR));
+            if (n <= 0)
+                n = sms / cs;
+            return std::min<long long>(n, sms / cs);
+        };
+        int R = 0, S = 0;
+        // static shared memory of the swapped kernel is a few hundred bytes: leave 1 KB for it
+        const int dyn_cap = info->smem_optin - 1024;
+        if (choose_swap(M, N, K, args.b_fp4 != 0, sms, dyn_cap, r_fixed, splits_override, capacity,
+                        R, S)) {
+            const int st_swap = launch_swap(args, dev, info, R, S, stages_override, timeout);
+            if (st_swap != DG_ERR_UNSUPPORTED || pair_mode == 4)
+                return st_swap;
+        } else if (pair_mode == 4) {
+            return DG_ERR_UNSUPPORTED;
+        }
+    }
+    if (pair_mode == 4)
+        pair_mode = 0;  // layouts and sizes the swapped kernel does not take run as in auto mode
     // Split-K clusters for dense problems with few output tiles (the memory-bound small-M
     // regime): auto mode uses them for M <= 256.
     if (args.layout == dg::kDense && (pair_mode == 3 || (pair_mode == 0 && M <= 256)) &&
@@ -1285,7 +1538,7 @@ int dg_set_pdl(int enable)
 
 int dg_set_kernel_family(int family)
 {
-    if (family < 0 || family > 3)
+    if (family < 0 || family > 4)
         return DG_ERR_INVALID_ARG;
     std::lock_guard<std::mutex> lock(g_mutex);
     int prev = g_family;

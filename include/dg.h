@@ -205,11 +205,15 @@ int dg_set_config_override(int block_n, int num_stages, int splits);
  * layout allows them (dense and masked; the contiguous layout always uses one-CTA tiles because
  * its expert segments are only 128-row aligned); 3 = the split-K cluster kernel for dense calls
  * whose output tiles fit in one wave (the K blocks of a tile are split over up to 8 CTAs that
- * reduce their fp32 partials through distributed shared memory, in a fixed order).  Automatic
- * mode uses split-K for dense M <= 256 when more than one split pays (else the one-CTA kernel),
- * pairs for dense M > 256 with K >= 96 * 128, and the one-CTA kernels otherwise (contiguous and
- * masked included).  Results agree within the parity tolerance whichever family runs.  Returns
- * the previous value, or DG_ERR_INVALID_ARG. */
+ * reduce their fp32 partials through distributed shared memory, in a fixed order); 4 = the
+ * swapped-operand kernel for dense calls with M <= 128 (B rows on the MMA's 128-row side, the
+ * tokens on its N side, K split over a cluster as in 3; block_n 128 or 256 of
+ * dg_set_config_override selects one or two 128-row blocks of B per tile), other calls run as
+ * in automatic mode.  Automatic mode uses the swapped-operand kernel for dense M <= 64 with one
+ * 128-row block of B per tile (when no block_n override is set), split-K for dense M <= 256 when
+ * more than one split pays (else the one-CTA kernel), pairs for dense M > 256 with
+ * K >= 96 * 128, and the one-CTA kernels otherwise (contiguous and masked included).  Results agree within the parity tolerance whichever
+ * family runs.  Returns the previous value, or DG_ERR_INVALID_ARG. */
 int dg_set_kernel_family(int family);
 
 /* Programmatic dependent launch (a Hopper/Blackwell launch feature, not on the pages; on by

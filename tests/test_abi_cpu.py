@@ -76,7 +76,8 @@ def test_config_override_validation(dg):
     assert dg.lib.dg_set_config_override(0, 0, 9) == dg.DG_ERR_INVALID_ARG
     assert dg.lib.dg_set_config_override(96, 4, 3) == dg.DG_OK
     assert dg.lib.dg_set_config_override(0, 0, 0) == dg.DG_OK
-    assert dg.lib.dg_set_kernel_family(4) == dg.DG_ERR_INVALID_ARG
+    assert dg.lib.dg_set_kernel_family(5) == dg.DG_ERR_INVALID_ARG
+    assert dg.lib.dg_set_kernel_family(4) == 0 and dg.lib.dg_set_kernel_family(0) == 4
     assert dg.lib.dg_set_fault_injection(2) == dg.DG_ERR_INVALID_ARG
     assert dg.lib.dg_set_fault_injection(0) == dg.DG_OK
     assert dg.lib.dg_set_kernel_family(0) == dg.DG_OK

@@ -76,7 +76,8 @@ def test_splitk_every_block_n(dg, orc, bn):
 
 
 def test_splitk_auto_selected_for_small_m(dg, orc):
-    case = workloads.dense(64, 4096, 7168, seed=71, a_std=1.0, b_std=0.02)
+    """Auto mode: 128 < M <= 256 runs split-K (M <= 128 takes the swapped-operand kernel)."""
+    case = workloads.dense(200, 4096, 7168, seed=71, a_std=1.0, b_std=0.02)
     _check(dg, orc, case, "auto small M")
     ll = dg.get_last_launch()
     assert ll["family"] == 3 and ll["splits"] > 1
@@ -98,7 +99,11 @@ def test_splitk_sm_cap(dg, orc):
 def test_splitk_deterministic(dg):
     """The reduction sums the partials in a fixed order: repeated calls are bit-identical."""
     case = workloads.dense(128, 2112, 7168, seed=73)
-    a = P.out_bits(P.run_dense(dg, case))
-    b = P.out_bits(P.run_dense(dg, case))
-    assert dg.get_last_launch()["splits"] > 1
+    dg.set_kernel_family(3)
+    try:
+        a = P.out_bits(P.run_dense(dg, case))
+        b = P.out_bits(P.run_dense(dg, case))
+        assert dg.get_last_launch()["splits"] > 1
+    finally:
+        dg.set_kernel_family(0)
     assert np.array_equal(a, b)

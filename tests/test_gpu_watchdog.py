@@ -40,6 +40,7 @@ def orc():
     (1, 1024, 2048, 4096),   # one-CTA persistent kernel
     (2, 1024, 2048, 4096),   # CTA-pair kernel
     (3, 128, 2048, 8192),    # split-K cluster kernel
+    (4, 64, 2048, 8192),     # swapped-operand kernel
 ])
 def test_wait_limit_reports_timeout_and_context_survives(dg, orc, family, M, N, K):
     case = workloads.dense(M, N, K, seed=family)
