@@ -53,7 +53,7 @@ SPEC_HBM_GBS = 8000.0     # B200 HBM3e bandwidth (data sheet)
 # profiles/).  `roofline.traffic` reports it; --traffic-bytes overrides it.  Re-measure after a
 # kernel change (a stale figure is worse than none).
 MEASURED_TRAFFIC = {
-    "dense 4096x7168x16384": 487783424 + 53111808,            # CTA pair BN 224
+    "dense 4096x7168x16384": 480949760 + 53178112,            # CTA pair BN 224
     "dg_quantize_1x128_kernel 8192x7168": 117451520 + 9024512,
     "dg_swiglu_quantize_1x128_kernel 16384x4096": 134243072 + 7325696,
 }
