@@ -9,13 +9,16 @@ Prints ONE JSON line on rank 0.  A "step" is one pass of the whole hot path over
 synthetic input: for the default workload, the fifteen GEMMs of the dense sweep
 (M in {64, 128, 4096} x (N, K) in {(2112,7168), (24576,1536), (7168,16384), (4096,7168),
 (7168,2048)}; A ~ N(0,1), B ~ N(0,0.02^2), fp32 scales per 1x128 tile of A and per 128x128
-block of B).  Inputs are resident in HBM; CUDA events bracket every GEMM on the launching
-stream, and the step is enqueued behind a bounded sleep kernel so that host latency never
-falls inside a bracket.  L2 is flushed (a 256 MiB write) before every step, and the step's own working set
-exceeds L2.
+block of B).  Inputs are resident in HBM.  Each timed step is one CUDA event pair on the
+launching stream around the step's GEMMs, enqueued back to back as a user would (programmatic
+dependent launch lets each kernel's set-up overlap the previous one's tail); the step is
+enqueued behind a bounded sleep kernel so that host latency never falls inside the bracket.  L2
+is flushed (a 256 MiB write) before every step, outside the bracket, and the step's own working
+set exceeds L2.  A second pass of the same steps brackets every GEMM with its own events for the
+per-shape figures and the roofline of the dominant kernel.
 
-`value` is the aggregate FP8 TFLOPS of the step (sum of 2*M*N*K over its GEMMs / sum of their
-device times), summed over ranks (each rank runs its own copy of the step: weak scaling, no
+`value` is the aggregate FP8 TFLOPS of the step (sum of 2*M*N*K over its GEMMs / device time of
+the step), summed over ranks (each rank runs its own copy of the step: weak scaling, no
 collective on the data path).  `e2e` is the same metric through the Python binding with host
 buffers: pinned host -> device copies of every input, the GEMMs, and the device -> host copy of
 every output inside the timed region.  `--impl reference` times the CPU oracle on a bounded
@@ -393,41 +396,65 @@ def run_ours(args, rank, world, local_rank):
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
     gate = [2_000_000]  # GPU cycles the stream is held so the host can enqueue the whole step
 
-    def step():
+    def gated(enqueue):
         # a bounded sleep kernel holds the stream while the host enqueues the step, so no host
-        # latency falls between an event and the GEMM it brackets; then the L2 flush
+        # latency falls inside an event bracket; then the L2 flush (outside the brackets)
         torch.cuda._sleep(gate[0])
         flush.fill_(1)
         t0 = time.perf_counter()
-        for i, d in enumerate(dev):
-            ev[i].record(stream)
-            d.launch(stream)
-        ev[n].record(stream)
+        enqueue()
         host = time.perf_counter() - t0
         stream.synchronize()
         if host * 1.9e9 * 1.5 > gate[0]:
             gate[0] = int(host * 1.9e9 * 3)
+
+    def step():
+        """One step as a user runs it: the GEMMs back to back, one event pair around them."""
+        def enqueue():
+            ev[0].record(stream)
+            for d in dev:
+                d.launch(stream)
+            ev[n].record(stream)
+        gated(enqueue)
+        return ev[0].elapsed_time(ev[n]) * 1e-3
+
+    def step_per_gemm():
+        """The same step with an event pair around every GEMM (per-shape and roofline figures;
+        the events between kernels cost each boundary its launch overlap)."""
+        def enqueue():
+            for i, d in enumerate(dev):
+                ev[i].record(stream)
+                d.launch(stream)
+            ev[n].record(stream)
+        gated(enqueue)
         return [ev[i].elapsed_time(ev[i + 1]) * 1e-3 for i in range(n)]
 
     for _ in range(args.warmup):
         step()
+        step_per_gemm()
     launch_info = dg.get_last_launch()
     if dg.poll_device_error(stream) != 0:
         raise RuntimeError("device error during warm-up")
 
-    per = [[] for _ in range(n)]
+    # the timed steps: whole-step device time
+    step_times = []
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
         for _ in range(args.steps):
-            for i, s in enumerate(step()):
-                per[i].append(s)
+            step_times.append(step())
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    total = sum(sum(p) for p in per)  # device seconds over the timed steps
+    total = sum(step_times)  # device seconds over the timed steps
     total_max = max_over_ranks(total, world, "cuda")
+
+    # per-GEMM breakdown (not part of `value`): the same number of steps with per-GEMM brackets
+    per = [[] for _ in range(n)]
+    for _ in range(args.steps):
+        for i, t in enumerate(step_per_gemm()):
+            per[i].append(t)
     if dg.poll_device_error(stream) != 0:
         raise RuntimeError("device error during the timed steps")
 
@@ -478,8 +505,12 @@ def run_ours(args, rank, world, local_rank):
                data="synthetic",
                config=dict(workload=desc, gemms_per_step=n,
                            l2="256 MiB write before every step; step working set > L2 (126 MB)",
-                           timing="CUDA events around each GEMM on the launching stream; the "
-                                  "step is enqueued behind a bounded sleep kernel",
+                           timing="value: one CUDA event pair per step on the launching stream "
+                                  "around the step's GEMMs enqueued back to back (programmatic "
+                                  "dependent launch on), the step enqueued behind a bounded sleep "
+                                  "kernel and the L2 flush outside the bracket; per_shape and "
+                                  "roofline: a second pass of the same steps with an event pair "
+                                  "around every GEMM",
                            parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
                gbs=world * bytes_step * args.steps / total_max / 1e9,
                roofline=roof, per_shape=shapes, back_to_back=b2b, gpu_launches=n * args.steps,
