@@ -64,3 +64,33 @@ def test_fp8_fp4_gemm_exact_rationals():
                     s += Fraction(oracle.e4m3_decode(int(a[m, k]))) * Fraction(oracle.e2m1_decode(nib))
                 exact += Fraction(float(sa[m, kb])) * Fraction(float(sb[0, kb])) * s
             assert abs(Fraction(float(res.acc[m, n])) - exact) <= Fraction(1, 10 ** 9) * (abs(exact) + 1)
+
+
+def test_grouped_expansion_is_per_group():
+    """The grouped FP8 x FP4 layouts pass B as [G, N, K/2]: the expansion of the whole array
+    equals the expansion of each group, and each code decodes to the nibble's E2M1 value."""
+    rng = np.random.default_rng(32)
+    G, N, K = 3, 5, 256
+    packed = rng.integers(0, 256, (G, N, K // 2), dtype=np.uint8)
+    whole = oracle.e2m1_to_e4m3(packed)
+    assert whole.shape == (G, N, K)
+    for g in range(G):
+        assert np.array_equal(whole[g], oracle.e2m1_to_e4m3(packed[g]))
+    g, n, k = 2, 4, 201
+    nib = (int(packed[g, n, k // 2]) >> 4) if (k & 1) else (int(packed[g, n, k // 2]) & 0xF)
+    assert oracle.e4m3_decode(int(whole[g, n, k])) == oracle.e2m1_decode(nib)
+
+
+def test_fp4_masked_gemm_equals_dense_per_group():
+    """A masked FP8 x FP4 GEMM computes, for each group, the dense GEMM of its valid rows."""
+    rng = np.random.default_rng(33)
+    G, M_max, N, K = 2, 4, 8, 256
+    a = rng.integers(0, 0x7E, (G, M_max, K), dtype=np.uint8)
+    sa = rng.uniform(0.5, 2.0, (G, M_max, K // 128)).astype(np.float32)
+    b = oracle.e2m1_to_e4m3(rng.integers(0, 256, (G, N, K // 2), dtype=np.uint8))
+    sb = rng.uniform(0.5, 2.0, (G, 1, K // 128)).astype(np.float32)
+    masked_m = np.array([3, 0], np.int32)
+    res = oracle.gemm_masked(a, sa, b, sb, masked_m)
+    dense = oracle.gemm_dense(a[0, :3], sa[0, :3], b[0], sb[0])
+    assert np.array_equal(res.bits[0, :3], dense.bits)
+    assert np.all(res.bits[0, 3:] == 0xFFFF) and np.all(res.bits[1] == 0xFFFF)
