@@ -84,6 +84,11 @@ def _load() -> ctypes.CDLL:
     lib.dg_swiglu_quantize_fp8_1x128.argtypes = [vp, vp, fp, i, i, ip, i, vp]
     lib.dg_swiglu_quantize_fp8_1x128.restype = i
     lib.dg_quantize_fp8_1x128.restype = i
+    lib.dg_set_tensor_map_cache.argtypes = [i]
+    lib.dg_set_tensor_map_cache.restype = i
+    lib.dg_get_tensor_map_cache_stats.argtypes = [ctypes.POINTER(ctypes.c_ulonglong),
+                                                  ctypes.POINTER(ctypes.c_ulonglong)]
+    lib.dg_get_tensor_map_cache_stats.restype = i
     lib.dg_set_pdl.argtypes = [i]
     lib.dg_set_pdl.restype = i
     ipp = ctypes.POINTER(ctypes.c_int)
@@ -220,6 +225,23 @@ def set_pdl(enable: bool) -> bool:
     if r < 0:
         raise DGError(r, "dg_set_pdl")
     return bool(r)
+
+
+def set_tensor_map_cache(enable: bool) -> bool:
+    """Turns the cache of encoded TMA tensor maps on or off (off drops every entry).  Returns
+    the previous setting."""
+    r = lib.dg_set_tensor_map_cache(1 if enable else 0)
+    if r < 0:
+        raise DGError(r, "dg_set_tensor_map_cache")
+    return bool(r)
+
+
+def tensor_map_cache_stats() -> tuple[int, int]:
+    """(hits, misses) of the tensor-map cache since the library was loaded."""
+    h, m = ctypes.c_ulonglong(), ctypes.c_ulonglong()
+    _check(lib.dg_get_tensor_map_cache_stats(ctypes.byref(h), ctypes.byref(m)),
+           "dg_get_tensor_map_cache_stats")
+    return h.value, m.value
 
 
 def get_last_launch() -> dict:

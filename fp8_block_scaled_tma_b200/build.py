@@ -11,7 +11,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdg_b200.so")
 SOURCES = ["dg_api.cu"]
-HEADERS = ["dg_kernel.cuh", "dg_pair_kernel.cuh", "dg_splitk_kernel.cuh", "dg_swap_kernel.cuh", "dg_quant_kernel.cuh",
+HEADERS = ["dg_kernel.cuh", "dg_map_cache.h", "dg_pair_kernel.cuh", "dg_splitk_kernel.cuh", "dg_swap_kernel.cuh",
+           "dg_quant_kernel.cuh",
            "dg_ptx.cuh"]
 
 NVCC_FLAGS = [

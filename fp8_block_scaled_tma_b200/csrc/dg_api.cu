@@ -12,6 +12,7 @@
 
 #include "../../include/dg.h"
 #include "dg_kernel.cuh"
+#include "dg_map_cache.h"
 #include "dg_pair_kernel.cuh"
 #include "dg_quant_kernel.cuh"
 #include "dg_splitk_kernel.cuh"
@@ -59,6 +60,7 @@ int g_pdl = 1;  // launch with programmatic stream serialisation (dg_set_pdl)
 // and kernel family; 0 = not queried yet
 int g_max_clusters[kMaxDevices][9][9];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+dg::TensorMapCache g_map_cache;  // encoded tensor maps, keyed on every encode argument
 
 struct LastLaunch {
     bool valid = false;
@@ -161,6 +163,20 @@ int align4(int x)
     return (x + 3) / 4 * 4;
 }
 
+// cuTensorMapEncodeTiled through the cache of encoded maps (a hit is byte-identical to what the
+// driver would encode for the same arguments).
+CUresult encode_tiled(CUtensorMap *map, CUtensorMapDataType dt, cuuint32_t rank, void *base,
+                      const cuuint64_t *dims, const cuuint64_t *strides, const cuuint32_t *box,
+                      const cuuint32_t *estr, CUtensorMapInterleave il, CUtensorMapSwizzle sw,
+                      CUtensorMapL2promotion l2, CUtensorMapFloatOOBfill oob)
+{
+    dg::TensorMapKey key;
+    dg::make_map_key(key, dt, rank, base, dims, strides, box, estr, il, sw, l2, oob);
+    return g_map_cache.get(key, map, [&](CUtensorMap *out) {
+        return g_encode(out, dt, rank, base, dims, strides, box, estr, il, sw, l2, oob);
+    });
+}
+
 // 3-D tiled tensor map: dims/strides innermost first (strides in bytes for dims 1, 2).
 int make_map(CUtensorMap *map, CUtensorMapDataType dt, void *base, uint64_t d0, uint64_t d1,
              uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1,
@@ -170,7 +186,7 @@ int make_map(CUtensorMap *map, CUtensorMapDataType dt, void *base, uint64_t d0, 
     cuuint64_t strides[2] = {stride1, stride2};
     cuuint32_t box[3] = {b0, b1, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = g_encode(map, dt, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+    CUresult r = encode_tiled(map, dt, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                           swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
@@ -188,7 +204,7 @@ int make_map_d(CUtensorMap *map, void *base, uint64_t N, uint64_t rows, int box_
     const CUtensorMapSwizzle swz = box_cols == 64   ? CU_TENSOR_MAP_SWIZZLE_128B
                                    : box_cols == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                     : CU_TENSOR_MAP_SWIZZLE_32B;
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+    CUresult r = encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? DG_OK : DG_ERR_CUDA;
@@ -214,7 +230,7 @@ int make_map_kblocks(CUtensorMap *map, void *base, uint64_t K, uint64_t rows, ui
     cuuint64_t strides[3] = {row_bytes, fp4 ? 64u : 128u, row_bytes * rows};
     cuuint32_t box[4] = {128, box_rows, kbs, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = g_encode(map, fp4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+    CUresult r = encode_tiled(map, fp4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8,
                           4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -1534,6 +1550,24 @@ int dg_set_pdl(int enable)
     int prev = g_pdl;
     g_pdl = enable;
     return prev;
+}
+
+int dg_set_tensor_map_cache(int enable)
+{
+    if (enable != 0 && enable != 1)
+        return DG_ERR_INVALID_ARG;
+    return g_map_cache.set_enabled(enable == 1) ? 1 : 0;
+}
+
+int dg_get_tensor_map_cache_stats(unsigned long long *hits, unsigned long long *misses)
+{
+    unsigned long long h = 0, m = 0;
+    g_map_cache.stats(h, m);
+    if (hits)
+        *hits = h;
+    if (misses)
+        *misses = m;
+    return DG_OK;
 }
 
 int dg_set_kernel_family(int family)

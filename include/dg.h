@@ -226,6 +226,18 @@ int dg_set_kernel_family(int family);
  * dependency).  enable: 0 or 1.  Returns the previous value, or DG_ERR_INVALID_ARG. */
 int dg_set_pdl(int enable);
 
+/* The cache of encoded TMA tensor maps (on by default).  Every GEMM call describes its operands
+ * with two to four tensor maps; an entry is keyed on every argument of the encoding (element
+ * type, base address, sizes, strides, box, swizzle, ...), so a hit is exactly the map that would
+ * be encoded and repeated calls on the same buffers skip the encoding.  enable 0 turns it off
+ * and drops every entry, 1 turns it on.  Returns the previous setting (0 or 1), or
+ * DG_ERR_INVALID_ARG.  Host-side only; thread-safe. */
+int dg_set_tensor_map_cache(int enable);
+
+/* Hits and misses of the tensor-map cache since the library was loaded (NULL pointers are
+ * skipped).  Returns DG_OK. */
+int dg_get_tensor_map_cache_stats(unsigned long long *hits, unsigned long long *misses);
+
 /* Describes the most recent launch on this host thread: fills any non-NULL pointer with the
  * chosen block_n, pipeline stages, grid size (CTAs), output tile count, kernel family (1, 2 or
  * 3 as in dg_set_kernel_family) and K splits per tile.  Returns DG_OK, or DG_ERR_INVALID_ARG

@@ -258,3 +258,34 @@ def test_masked_out_of_range_count_reports_layout_error(dg):
 
 def test_no_device_error_left(dg):
     assert dg.poll_device_error() == 0
+
+
+def test_tensor_map_cache_hits_and_matches_uncached(dg, orc):
+    """Repeated calls on the same buffers reuse their encoded tensor maps, and the results are
+    bit-identical with the cache on and off (and match the oracle)."""
+    case = workloads.dense(200, 1000, 640, seed=801)
+    a, b = P.to_dev_u8(case.a), P.to_dev_u8(case.b)
+    sfa, sfb = dg.sfa_mn_major(P.to_dev_f32(case.sa)), P.to_dev_f32(case.sb)
+    d = P.sentinel_out((case.M, case.N))
+    dg.dg_gemm_fp8_fp8_bf16_nt(a, sfa, b, sfb, d)
+    torch.cuda.synchronize()
+    first = P.out_bits(d)
+    h0, m0 = dg.tensor_map_cache_stats()
+    for _ in range(3):
+        dg.dg_gemm_fp8_fp8_bf16_nt(a, sfa, b, sfb, d)
+    torch.cuda.synchronize()
+    h1, m1 = dg.tensor_map_cache_stats()
+    assert h1 - h0 >= 6 and m1 == m0, (h0, m0, h1, m1)
+    assert np.array_equal(P.out_bits(d), first)
+    prev = dg.set_tensor_map_cache(False)
+    try:
+        d.view(torch.int16).fill_(-1)
+        dg.dg_gemm_fp8_fp8_bf16_nt(a, sfa, b, sfb, d)
+        torch.cuda.synchronize()
+        uncached = P.out_bits(d)
+    finally:
+        dg.set_tensor_map_cache(prev)
+    assert np.array_equal(uncached, first)
+    ref = orc.gemm_dense(case.a, case.sa, case.b, case.sb)
+    P.assert_close(first, ref.bits, ref.mag, "cached maps")
+    assert dg.poll_device_error() == 0
