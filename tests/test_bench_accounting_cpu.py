@@ -1,0 +1,65 @@
+"""The algorithmic FLOP and byte counts behind bench.py's roofline fractions, checked on small
+cases against the definitions written out by hand: each operand once, the rows that are
+computed (contiguous: valid rows; masked: rows below masked_m), the groups touched, an FP4 B at
+half a byte per element, and t_roof = max(FLOPs / P_fp8, bytes / BW)."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import bench
+import workloads
+
+
+def test_dense_counts():
+    c = workloads.dense(64, 256, 384, seed=1)
+    g = bench.Gemm("dense", c, "d")
+    assert g.flops == 2.0 * 64 * 256 * 384
+    kb, nb = 3, 2
+    assert g.bytes == 64 * 384 + 256 * 384 + 2 * 64 * 256 + 4 * 64 * kb + 4 * nb * kb
+
+
+def test_dense_fp4_halves_b():
+    c = workloads.dense(64, 256, 384, seed=1)
+    g8 = bench.Gemm("dense", c, "d")
+    g4 = bench.Gemm("dense", workloads.with_fp4_b(c, seed=2), "d fp4", fp4=True)
+    assert g8.flops == g4.flops
+    assert g8.bytes - g4.bytes == 256 * 384 // 2
+
+
+def test_contiguous_counts_valid_rows_and_touched_groups():
+    c = workloads.contiguous(G=4, N=128, K=256, seed=3, counts=[5, 0, 130, 128])
+    g = bench.Gemm("contiguous", c, "c")
+    m_valid = 5 + 130 + 128
+    m_rows = c.M_total                       # 128 + 0 + 256 + 128 = 512
+    assert m_rows == 512
+    assert g.flops == 2.0 * m_valid * 128 * 256
+    kb = 2
+    assert g.bytes == (m_valid * 256 + 128 * 256 * 3 + 2 * m_valid * 128 + 4 * m_rows * kb
+                       + 4 * 1 * kb * 3 + 4 * m_rows)
+
+
+def test_masked_counts_rows_below_masked_m():
+    c = workloads.masked(G=3, M_max=64, N=256, K=128, seed=4, masked_m=[10, 0, 64])
+    g = bench.Gemm("masked", c, "m")
+    assert g.flops == 2.0 * 74 * 256 * 128
+    assert g.bytes == 74 * 128 + 256 * 128 * 2 + 2 * 74 * 256 + 4 * 74 * 1 + 4 * 2 * 1 * 2
+
+
+def test_roofline_bound_and_fraction():
+    c = workloads.dense(4096, 4096, 4096, seed=5)
+    g = bench.Gemm("dense", c, "big")
+    peaks = dict(hbm_gbs=6000.0, bf16_tflops=1500.0, bf16_tflops_sustained=1400.0, source="test")
+    p_fp8 = 1500.0 * bench.FP8_PER_BF16 * 1e12
+    t_roof = max(g.flops / p_fp8, g.bytes / 6000e9)
+    r = bench.roofline(g, 2 * t_roof, peaks)
+    assert r["bound"] == "tensor"
+    assert r["frac"] == pytest.approx(0.5)
+    assert r["tflops"] == pytest.approx(g.flops / (2 * t_roof) / 1e12)
+    small = bench.Gemm("dense", workloads.dense(64, 4096, 4096, seed=6), "small")
+    assert bench.roofline(small, 1e-3, peaks)["bound"] == "hbm"
+
+
+def test_quant_and_swiglu_bytes():
+    assert bench.quant_bytes(8, 256) == 8 * 256 * 2 + 8 * 256 + 4 * 8 * 2
+    assert bench.swiglu_bytes(8, 256) == 8 * 512 * 2 + 8 * 256 + 4 * 8 * 2
