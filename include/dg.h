@@ -69,7 +69,7 @@ int dg_gemm_fp8_fp8_bf16_nt(const void *a, const float *sfa, const void *b, cons
  * M_total must be a multiple of 128 and every aligned 128-row tile may hold rows of one
  * expert only (plus -1 rows): the segments of each expert are padded to 128 rows.  A tile
  * that breaks this, or an index outside [-1, G), sets DG_ERR_LAYOUT on the device and the
- * offending rows are not written. */
+ * offending rows are not written.  G >= 1; M_total == 0 is a no-op. */
 int dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(const void *a, const float *sfa, const void *b,
                                                  const float *sfb, void *d, const int *m_indices,
                                                  int M_total, int N, int K, int G,
@@ -87,7 +87,9 @@ int dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(const void *a, const float *sfa
  *              clamped.
  *   expected_m host-side hint of the typical masked_m (used only to choose tiles; never
  *              changes results).  masked_m is read on the device only, so the call needs no
- *              host synchronisation. */
+ *              host synchronisation.
+ * 1 <= G <= 1024 (the device-side tile scheduler keeps a prefix sum per group), M_max >= 0
+ * (M_max == 0 is a no-op), expected_m >= 0; DG_ERR_INVALID_ARG otherwise. */
 int dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked(const void *a, const float *sfa, const void *b,
                                              const float *sfb, void *d, const int *masked_m,
                                              int G, int M_max, int N, int K, int expected_m,
