@@ -131,6 +131,14 @@ def test_grouped_reject_bad_arguments(dg):
                                                       256, 256, 128, None, 0, None) == -1
 
 
+def test_masked_group_limit(dg):
+    L = dg.lib
+    assert L.dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1025,
+                                                      128, 256, 256, 64, None, 0, None) == -1
+    assert L.dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1024,
+                                                      0, 256, 256, 64, None, 0, None) == 0
+
+
 def test_fp4_entries_reject_bad_arguments(dg):
     L = dg.lib
     # packed E2M1 B must be 32-byte aligned (16 is enough for e4m3 B)
