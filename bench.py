@@ -6,10 +6,17 @@
                     [--fp4]
 
 Prints ONE JSON line on rank 0.  A "step" is one pass of the whole hot path over one batch of
-synthetic input: for the default workload, the fifteen GEMMs of the dense sweep
-(M in {64, 128, 4096} x (N, K) in {(2112,7168), (24576,1536), (7168,16384), (4096,7168),
-(7168,2048)}; A ~ N(0,1), B ~ N(0,0.02^2), fp32 scales per 1x128 tile of A and per 128x128
-block of B).  Inputs are resident in HBM.  Each timed step is one CUDA event pair on the
+synthetic input: for the default workload ("all"), the nineteen GEMMs of the five workload
+configurations, each GEMM once:
+  1. dense 128 x 256 x 512, A and B ~ N(0,1);
+  2. the dense sweep, M in {64, 128, 4096} x (N, K) in {(2112,7168), (24576,1536),
+     (7168,16384), (4096,7168), (7168,2048)}, A ~ N(0,1), B ~ N(0,0.02^2) (15 GEMMs);
+  3. the contiguous grouped MoE GEMM, G = 8, per-expert counts U[128, 1024] padded to 128,
+     N = 4096, K = 7168;
+  4. the masked grouped MoE GEMM, G = 32, M_max = 256, masked_m U[0, 256], N = 4096, K = 7168;
+  5. the prefill GEMM 8192 x 7168 x 18432 with 1 % x50 outliers in A;
+all with fp32 scales per 1x128 tile of A and per 128x128 block of B.  `per_shape` has one
+entry per GEMM and `per_config` one per configuration.  Inputs are resident in HBM.  Each timed step is one CUDA event pair on the
 launching stream around the step's GEMMs, enqueued back to back as a user would (programmatic
 dependent launch lets each kernel's set-up overlap the previous one's tail); the step is
 enqueued behind a bounded sleep kernel so that host latency never falls inside the bracket.  L2
@@ -52,14 +59,39 @@ SPEC_FP8_TFLOPS = 4500.0  # B200 dense FP8 tensor peak (data sheet)
 SPEC_HBM_GBS = 8000.0     # B200 HBM3e bandwidth (data sheet)
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernel
-# of each default workload, from one ncu capture of the current kernels (summaries under
-# profiles/).  `roofline.traffic` reports it; --traffic-bytes overrides it.  Re-measure after a
-# kernel change (a stale figure is worse than none).
+# of a workload, from one ncu capture (summaries under profiles/), with the fingerprint of the
+# kernel sources it was taken on (`kernel_source_fingerprint`).  `roofline.traffic` reports the
+# figure only while the sources still have that fingerprint, and null once a kernel changed
+# since the counters were taken; --traffic-bytes overrides it.
 MEASURED_TRAFFIC = {
-    "dense 4096x7168x16384": 480949760 + 53178112,            # CTA pair BN 224
-    "dg_quantize_1x128_kernel 8192x7168": 117451520 + 9024512,
-    "dg_swiglu_quantize_1x128_kernel 16384x4096": 134243072 + 7325696,
+    "dg_quantize_1x128_kernel 8192x7168": (117451520 + 9024512, None),
+    "dg_swiglu_quantize_1x128_kernel 16384x4096": (134243072 + 7325696, None),
 }
+
+
+def kernel_source_fingerprint() -> str:
+    """sha256 (first 16 hex digits) of the library's CUDA sources and its header."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "fp8_block_scaled_tma_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    with open(os.path.join(ROOT, "include", "dg.h"), "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(name: str, override=None):
+    """(bytes per launch or None, note) for the dominant kernel `name`."""
+    if override:
+        return override, "--traffic-bytes"
+    if name not in MEASURED_TRAFFIC:
+        return None, "no ncu capture of this kernel"
+    value, fp = MEASURED_TRAFFIC[name]
+    if fp is not None and fp != kernel_source_fingerprint():
+        return None, "the kernel sources changed since the ncu capture"
+    return value, f"ncu capture, kernel sources {fp or 'not fingerprinted'}"
 
 
 # ---- workload description ---------------------------------------------------------------------
@@ -67,8 +99,8 @@ MEASURED_TRAFFIC = {
 class Gemm:
     """One GEMM of a step: its kind, sizes, FLOPs and algorithmic bytes."""
 
-    def __init__(self, kind: str, case, name: str, fp4: bool = False):
-        self.kind, self.case, self.name, self.fp4 = kind, case, name, fp4
+    def __init__(self, kind: str, case, name: str, fp4: bool = False, config: int = 0):
+        self.kind, self.case, self.name, self.fp4, self.config = kind, case, name, fp4, config
         self._oracle_b = None
         c = case
         if kind == "dense":
@@ -90,6 +122,8 @@ class Gemm:
         self.bytes = (m_valid * K + b_bytes + 2 * m_valid * N + 4 * m_rows * kb
                       + 4 * nb * kb * groups + (4 * M if kind == "contiguous" else 0))
         self.shape = dict(kind=kind, M=M, N=N, K=K, G=getattr(c, "G", 1), M_valid=m_valid)
+        if config:
+            self.shape["config"] = config
 
     def oracle_b(self):
         """B as the oracle takes it: e4m3 codes (an FP4 B expanded once by the oracle)."""
@@ -109,12 +143,28 @@ def build_workload(name: str, shape=None, fp4: bool = False):
         return gemms, desc
     out = []
     for i, g in enumerate(gemms):
-        out.append(Gemm(g.kind, workloads.with_fp4_b(g.case, seed=7000 + i), g.name + " fp4", fp4=True))
+        out.append(Gemm(g.kind, workloads.with_fp4_b(g.case, seed=7000 + i), g.name + " fp4", fp4=True,
+                        config=g.config))
     return out, desc.replace("B~N(0,0.02)", "B packed FP4 E2M1 (uniform codes, 128x128 fp32 block scales)") \
         + "; FP8 x FP4"
 
 
+CONFIG_NAMES = {1: "dense 128x256x512", 2: "dense sweep (15 shapes)", 3: "contiguous G=8",
+                4: "masked G=32", 5: "prefill 8192x7168x18432"}
+
+
 def _build_workload(name: str, shape=None):
+    if name == "all":
+        parts = [("small", 1), ("sweep", 2), ("contiguous", 3), ("masked", 4), ("prefill", 5)]
+        gemms, descs = [], []
+        for part, cfg in parts:
+            gs, d = _build_workload(part)
+            for g in gs:
+                g.config = cfg
+                g.shape["config"] = cfg
+            gemms += gs
+            descs.append(f"({cfg}) {d}")
+        return gemms, "the five configurations, each GEMM once per step: " + "; ".join(descs)
     if name == "dense":
         M, N, K = shape
         c = workloads.dense(M, N, K, seed=6000, a_std=1.0, b_std=0.02)
@@ -490,10 +540,10 @@ def run_ours(args, rank, world, local_rank):
         peak = peaks["hbm_gbs"]
         roof = dict(bound="hbm", achieved=dsh["gbs"], peak=peak, unit="GB/s",
                     frac=dsh["gbs"] / peak, peak_source=f"{peaks['source']} HBM copy")
-    roof.update(kernel=dsh["name"],
-                traffic=args.traffic_bytes if args.traffic_bytes else MEASURED_TRAFFIC.get(dsh["name"]),
-                traffic_unit="bytes/launch",
-                frac_spec=dsh["frac_spec"])
+    traffic, traffic_note = measured_traffic(dsh["name"], args.traffic_bytes)
+    roof.update(kernel=dsh["name"], traffic=traffic, traffic_unit="bytes/launch",
+                traffic_source=traffic_note, frac_spec=dsh["frac_spec"],
+                launches_timed=args.steps)
     if rank == 0 and not args.no_cublas:
         # context only: what cuBLAS reaches on an FP8 GEMM on this GPU
         roof["cublas_fp8_tflops_8192"] = measure_cublas_fp8()
@@ -503,17 +553,10 @@ def run_ours(args, rank, world, local_rank):
                higher_is_better=True, scaling="weak", vs_baseline=None,
                dtype="e4m3 x e2m1 -> f32" if args.fp4 else "e4m3 x e4m3 -> f32",
                data="synthetic",
-               config=dict(workload=desc, gemms_per_step=n,
-                           l2="256 MiB write before every step; step working set > L2 (126 MB)",
-                           timing="value: one CUDA event pair per step on the launching stream "
-                                  "around the step's GEMMs enqueued back to back (programmatic "
-                                  "dependent launch on), the step enqueued behind a bounded sleep "
-                                  "kernel and the L2 flush outside the bracket; per_shape and "
-                                  "roofline: a second pass of the same steps with an event pair "
-                                  "around every GEMM",
-                           parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+               config=bench_config(desc, n, world),
                gbs=world * bytes_step * args.steps / total_max / 1e9,
-               roofline=roof, per_shape=shapes, back_to_back=b2b, gpu_launches=n * args.steps,
+               roofline=roof, per_shape=shapes, per_config=per_config(shapes),
+               back_to_back=b2b, gpu_launches=n * args.steps,
                clocks=clk.summary(), last_launch=launch_info)
 
     # e2e through the public API with host buffers
@@ -521,6 +564,39 @@ def run_ours(args, rank, world, local_rank):
         out["e2e"] = run_e2e(dg, dev, gemms, args, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(gemms, budget_s=args.cpu_seconds)
+    return out
+
+
+def bench_config(desc: str, n_gemms: int, world: int) -> dict:
+    """The `config` of the JSON line; both arms print the same one for a workload."""
+    return dict(workload=desc, gemms_per_step=n_gemms,
+                l2="256 MiB write before every step; step working set > L2 (126 MB)",
+                timing="value: one CUDA event pair per step on the launching stream around the "
+                       "step's GEMMs enqueued back to back (programmatic dependent launch on), the "
+                       "step enqueued behind a bounded sleep kernel and the L2 flush outside the "
+                       "bracket; per_shape and roofline: a second pass of the same steps with an "
+                       "event pair around every GEMM",
+                parallelism=f"replicas x{world}" if world > 1 else "single GPU")
+
+
+def per_config(shapes) -> list:
+    """Per workload configuration: its GEMMs' summed event times, TFLOPS and algorithmic GB/s,
+    and the fraction of its roofline (summed roofline time / summed time), also in a CUDA
+    graph where every GEMM of the configuration has a graph time."""
+    out = []
+    for cfg in sorted({sh.get("config", 0) for sh in shapes}):
+        sel = [sh for sh in shapes if sh.get("config", 0) == cfg]
+        us = sum(sh["us"] for sh in sel)
+        roof = sum(sh["roof_us"] for sh in sel)
+        flops = sum(sh["tflops"] * sh["us"] for sh in sel)   # TFLOPS x us = MFLOP
+        gb = sum(sh["gbs"] * sh["us"] for sh in sel)
+        e = dict(config=cfg, name=CONFIG_NAMES.get(cfg, "workload"), gemms=len(sel), us=us,
+                 tflops=flops / us, gbs=gb / us, frac=roof / us,
+                 bound=sorted({sh["bound"] for sh in sel}))
+        if all("graph_us" in sh for sh in sel):
+            g = sum(sh["graph_us"] for sh in sel)
+            e.update(graph_us=g, graph_frac=roof / g if g > 0 else None)
+        out.append(e)
     return out
 
 
@@ -665,7 +741,7 @@ def run_reference(args):
     return dict(metric=METRIC, value=value, unit=UNIT, n_gpus=1, steps=args.steps,
                 warmup=args.warmup, ms_per_step=dt / args.steps * 1e3, higher_is_better=True,
                 scaling="weak", vs_baseline=None, dtype="f64", data="synthetic",
-                config=dict(workload=desc), impl="reference",
+                config=bench_config(desc, len(gemms), 1), impl="reference",
                 cpu_baseline=dict(value=value, unit=UNIT, cores=cores, kind="oracle", sample=sample),
                 e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
 
@@ -754,7 +830,7 @@ def run_quant(args, rank, world, local_rank):
                 kernel=(f"dg_swiglu_quantize_1x128_kernel {M}x{2 * K}" if swiglu
                         else f"dg_quantize_1x128_kernel {M}x{K}"),
                 traffic_unit="bytes/launch")
-    roof["traffic"] = args.traffic_bytes if args.traffic_bytes else MEASURED_TRAFFIC.get(roof["kernel"])
+    roof["traffic"], roof["traffic_source"] = measured_traffic(roof["kernel"], args.traffic_bytes)
     # e2e: pinned host bf16 in, quantise, codes and scales out
     hx = x.cpu().pin_memory()
     hq = torch.empty_like(q, device="cpu").pin_memory()
@@ -813,7 +889,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["sweep", "small", "contiguous", "masked", "prefill",
-                                           "dense", "quant", "swiglu"], default="sweep")
+                                           "dense", "quant", "swiglu", "all"], default="all")
     ap.add_argument("--shape", type=lambda v: tuple(int(x) for x in v.split(",")), default=None,
                     help="M,N,K of --workload dense; M,K of --workload quant; M,I of --workload swiglu")
     ap.add_argument("--block-n", type=int, default=0, help="tile override (tuning)")

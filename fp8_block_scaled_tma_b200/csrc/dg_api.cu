@@ -27,6 +27,14 @@ constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
 constexpr int kMinDynSmem = 120 * 1024;  // keeps one CTA per SM (each takes all 512 TMEM columns)
 
 __device__ int g_device_error;  // the device error word read by dg_poll_device_error
+__device__ int g_polled_error;  // the value dg_poll_device_error last took from it
+
+// Takes the error word and resets it in one atomic step, so that no error recorded by a
+// kernel running on another stream can fall between the read and the reset.
+__global__ void dg_take_error_kernel()
+{
+    g_polled_error = atomicExch(&g_device_error, 0);
+}
 
 struct DeviceInfo {
     bool init = false;
@@ -1499,9 +1507,10 @@ int dg_poll_device_error(void *stream)
         return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int value = 0;
-    const int zero = 0;
-    if (cudaMemcpyAsync(&value, info->err_ptr, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaMemcpyAsync(info->err_ptr, &zero, sizeof(int), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+    dg_take_error_kernel<<<1, 1, 0, s>>>();
+    if (cudaGetLastError() != cudaSuccess ||
+        cudaMemcpyFromSymbolAsync(&value, g_polled_error, sizeof(int), 0, cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess) {
         cudaGetLastError();
         return DG_ERR_CUDA;

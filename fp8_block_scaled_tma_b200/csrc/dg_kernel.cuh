@@ -160,11 +160,18 @@ __device__ __forceinline__ bool resolve_tile(const Params &p, const SmemCtl &ctl
         ti.a_z = 0;
         ti.g = 0;
         if (L == kContiguous) {
+            // the tile's expert is that of its first non-padding row; an index below -1 breaks
+            // the layout contract (reported, and the row is treated as padding: not written)
             int g = __ldg(p.m_indices + ti.m0);
+            if (g < -1)
+                record_error(p.err, kErrLayout);
             if (g < 0) {
                 int end = ti.m0 + kBlockM < p.M ? ti.m0 + kBlockM : p.M;
-                for (int r2 = ti.m0 + 1; r2 < end && g < 0; ++r2)
+                for (int r2 = ti.m0 + 1; r2 < end && g < 0; ++r2) {
                     g = __ldg(p.m_indices + r2);
+                    if (g < -1)
+                        record_error(p.err, kErrLayout);
+                }
             }
             if (g < 0)
                 return false;          // an all-padding tile: nothing to write
@@ -774,7 +781,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 if (grow < p.M) {
                     const int gi = __ldg(p.m_indices + grow);
                     valid = gi == ti.g;
-                    if (gi >= 0 && gi != ti.g)
+                    if ((gi >= 0 && gi != ti.g) || gi < -1)
                         record_error(p.err, kErrLayout);
                 }
                 out_row = static_cast<size_t>(grow);

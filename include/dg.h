@@ -180,8 +180,13 @@ size_t dg_get_workspace_size(int kind, int M, int N, int K, int G);
 const char *dg_status_string(int status);
 
 /* Reads the device error word that contract checks and the pipeline watchdog set, resets it
- * to 0, and returns it (DG_OK, DG_ERR_TIMEOUT or DG_ERR_LAYOUT).  This call SYNCHRONISES
- * `stream`; it is meant for tests and debugging, not for the hot path. */
+ * to 0, and returns it (DG_OK, DG_ERR_TIMEOUT or DG_ERR_LAYOUT).  The read and the reset are
+ * one atomic exchange on the device, enqueued on `stream`.  There is ONE word per device,
+ * shared by the kernels of every stream and thread: an error is seen by the first poll that
+ * runs after the kernel recorded it, whichever stream that poll is on, and a kernel still
+ * running on another stream may record its error after this poll (synchronise the device, or
+ * every stream that ran this library's kernels, before polling to see them all).  This call
+ * SYNCHRONISES `stream`; it is meant for tests and debugging, not for the hot path. */
 int dg_poll_device_error(void *stream);
 
 /* Time limit, in nanoseconds, of every pipeline wait inside the kernels (default 2e9).

@@ -5,6 +5,13 @@ Tolerance (per element, on valid rows):  |D - Dref| <= 2 * ulp_bf16(Dref) + 1e-3
 with ulp_bf16(x) = 2^(max(floor(log2 |x|), -126) - 7) (2^-133 for x = 0); and per matrix
 1 - 2<D,Dref> / (<D,D> + <Dref,Dref>) <= 1e-5 in fp64.  Rows the call must not write keep the
 sentinel bit pattern exactly.
+
+Every comparison also bounds the error beyond the final bf16 rounding ("excess", see
+``compare``) by 1e-5 of sum_k |sa a| |sb b|.  That is what fp32 accumulation of the 128-wide
+K-slice partials allows (one fp32 rounding per slice and per promotion: at most about
+(K/128 + 1) * 2^-24 relative to the magnitude, 8.6e-6 at K = 18432), and what an accumulator
+of fewer bits -- the FP8 tensor-core imprecision that two-level accumulation exists to contain
+(DeepGEMM release write-up, "深入了解DeepGEMM") -- would exceed.
 """
 from __future__ import annotations
 
@@ -15,6 +22,7 @@ SENTINEL = 0xFFFF  # a bf16 NaN pattern no finite result can take
 ULP_FACTOR = 2.0
 MAG_FACTOR = 1e-3
 DIFF_MAX = 1e-5
+EXCESS_MAX = 1e-5
 
 
 def bits_to_f64(bits: np.ndarray) -> np.ndarray:
@@ -50,11 +58,23 @@ def compare(got_bits: np.ndarray, ref_bits: np.ndarray, mag: np.ndarray, acc=Non
                 first_bad=None if not bad.any() else tuple(int(i) for i in np.argwhere(bad)[0]))
 
 
-def assert_close(got_bits, ref_bits, mag, what: str = "", acc=None) -> dict:
+def assert_close(got_bits, ref_bits, mag, what: str, acc) -> dict:
+    """The parity bar: every element within tolerance, the matrix difference within DIFF_MAX,
+    and the error beyond one bf16 rounding within EXCESS_MAX of the magnitude.  ``acc`` is the
+    oracle's unrounded fp64 result for the same entries (required)."""
     r = compare(got_bits, ref_bits, mag, acc)
     assert r["n_bad"] == 0, f"{what}: {r['n_bad']}/{r['n']} elements out of tolerance, first at {r['first_bad']}: {r}"
     assert r["diff"] <= DIFF_MAX, f"{what}: matrix diff {r['diff']} > {DIFF_MAX}"
+    assert r["excess"] < EXCESS_MAX, f"{what}: error beyond one bf16 rounding {r['excess']} >= {EXCESS_MAX}"
     return r
+
+
+def check(got_bits, ref, what: str, sel=None) -> dict:
+    """assert_close against an oracle Result, optionally on a selection ``sel`` (an index or
+    mask applied alike to the GPU bits and to the oracle's arrays)."""
+    if sel is None:
+        return assert_close(got_bits, ref.bits, ref.mag, what, ref.acc)
+    return assert_close(got_bits[sel], ref.bits[sel], ref.mag[sel], what, ref.acc[sel])
 
 
 def to_dev_u8(x: np.ndarray) -> torch.Tensor:
@@ -148,10 +168,28 @@ def run_masked_fp4(dg, case) -> torch.Tensor:
 
 
 def sample_rows(M: int, n: int, seed: int) -> np.ndarray:
-    """Rows at tile boundaries (first/last rows of the first, second and last 128-row tiles)
-    plus n seeded random rows."""
+    """Rows at tile boundaries (first/last rows of the first, second and last 128-row tiles),
+    one seeded row in EVERY 128-row tile (so that a tile written to the wrong place, or not
+    at all, cannot hide between samples), plus n seeded random rows."""
     rng = np.random.default_rng(seed)
     fixed = [0, 1, 127, 128, 129, 255, M - 129, M - 128, M - 2, M - 1]
     rows = set(r for r in fixed if 0 <= r < M)
+    for t0 in range(0, M, 128):
+        rows.add(int(rng.integers(t0, min(t0 + 128, M))))
     rows.update(int(r) for r in rng.integers(0, M, size=min(n, M)))
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def sample_valid_rows(valid: np.ndarray, n: int, seed: int) -> np.ndarray:
+    """For a grouped layout with a per-row validity mask: the first and last valid rows, one
+    seeded valid row in every 128-row tile that has one, plus n seeded valid rows."""
+    rng = np.random.default_rng(seed)
+    idx = np.nonzero(valid)[0]
+    rows = set(int(r) for r in idx[:2]) | set(int(r) for r in idx[-2:])
+    for t0 in range(0, len(valid), 128):
+        v = idx[(idx >= t0) & (idx < t0 + 128)]
+        if v.size:
+            rows.add(int(rng.choice(v)))
+    if idx.size:
+        rows.update(int(r) for r in rng.choice(idx, size=min(n, idx.size), replace=False))
     return np.array(sorted(rows), dtype=np.int64)

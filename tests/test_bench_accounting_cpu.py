@@ -63,3 +63,30 @@ def test_roofline_bound_and_fraction():
 def test_quant_and_swiglu_bytes():
     assert bench.quant_bytes(8, 256) == 8 * 256 * 2 + 8 * 256 + 4 * 8 * 2
     assert bench.swiglu_bytes(8, 256) == 8 * 512 * 2 + 8 * 256 + 4 * 8 * 2
+
+
+def test_per_config_sums_times_and_roofline():
+    """per_config: TFLOPS and GB/s over a configuration's summed times, and the fraction as
+    summed roofline time over summed time (graph fraction only when every GEMM has one)."""
+    shapes = [
+        dict(config=2, us=10.0, roof_us=5.0, tflops=1.0, gbs=100.0, bound="hbm", graph_us=8.0),
+        dict(config=2, us=30.0, roof_us=15.0, tflops=3.0, gbs=300.0, bound="tensor"),
+        dict(config=4, us=20.0, roof_us=16.0, tflops=2.0, gbs=500.0, bound="hbm", graph_us=18.0),
+    ]
+    pc = {e["config"]: e for e in bench.per_config(shapes)}
+    assert pc[2]["us"] == 40.0 and pc[2]["frac"] == pytest.approx(0.5)
+    assert pc[2]["tflops"] == pytest.approx((10 * 1.0 + 30 * 3.0) / 40)
+    assert pc[2]["gbs"] == pytest.approx((10 * 100 + 30 * 300) / 40)
+    assert "graph_frac" not in pc[2] and pc[2]["bound"] == ["hbm", "tensor"]
+    assert pc[4]["graph_frac"] == pytest.approx(16.0 / 18.0)
+
+
+def test_traffic_reported_only_for_unchanged_kernel_sources(monkeypatch):
+    fp = bench.kernel_source_fingerprint()
+    assert len(fp) == 16 and fp == bench.kernel_source_fingerprint()
+    monkeypatch.setitem(bench.MEASURED_TRAFFIC, "k same", (123, fp))
+    monkeypatch.setitem(bench.MEASURED_TRAFFIC, "k stale", (456, "0" * 16))
+    assert bench.measured_traffic("k same")[0] == 123
+    assert bench.measured_traffic("k stale")[0] is None
+    assert bench.measured_traffic("k unknown")[0] is None
+    assert bench.measured_traffic("k stale", 789)[0] == 789

@@ -104,8 +104,8 @@ def test_fp4_equals_fp8_of_same_values(dg, orc):
     case8 = dataclasses.replace(case, b=orc.e2m1_to_e4m3(case.b))
     got8 = P.out_bits(P.run_dense(dg, case8))
     ref = orc.gemm_dense(case8.a, case8.sa, case8.b, case8.sb)
-    P.assert_close(got4, ref.bits, ref.mag, "fp4")
-    P.assert_close(got8, ref.bits, ref.mag, "fp8 of the same values")
+    P.check(got4, ref, "fp4")
+    P.check(got8, ref, "fp8 of the same values")
     assert np.mean(got4 == got8) > 0.99
 
 
@@ -115,7 +115,7 @@ def test_fp4_decode_and_prefill_shapes_sampled(dg, orc, M):
     on sampled rows."""
     for N, K in [(7168, 2048), (2112, 7168)]:
         case = workloads.with_fp4_b(workloads.dense(M, N, K, seed=M + N), seed=K)
-        rows = P.sample_rows(M, 24, seed=M)
+        rows = P.sample_rows(M, 8, seed=M)
         _dense(dg, orc, case, f"fp4 {M}x{N}x{K}", rows=rows)
 
 
@@ -126,7 +126,7 @@ def test_fp4_contiguous(dg, orc):
     ref = orc.gemm_contiguous(case.a, case.sa, orc.e2m1_to_e4m3(case.b), case.sb, case.m_indices)
     pad = case.m_indices < 0
     assert np.all(got[pad] == P.SENTINEL), "a padding row was written"
-    P.assert_close(got[~pad], ref.bits[~pad], ref.mag[~pad], "fp4 contiguous")
+    P.check(got, ref, "fp4 contiguous", sel=~pad)
     assert dg.poll_device_error() == 0
 
 
@@ -143,7 +143,7 @@ def test_fp4_masked(dg, orc, family):
     ref = orc.gemm_masked(case.a, case.sa, orc.e2m1_to_e4m3(case.b), case.sb, case.masked_m)
     inv = np.arange(case.M_max)[None, :] >= case.masked_m[:, None]
     assert np.all(got[inv] == P.SENTINEL), "a row beyond masked_m was written"
-    P.assert_close(got[~inv], ref.bits[~inv], ref.mag[~inv], f"fp4 masked family {family}")
+    P.check(got, ref, f"fp4 masked family {family}", sel=~inv)
     assert dg.poll_device_error() == 0
 
 

@@ -112,7 +112,7 @@ def test_dense_sweep_full_size_sampled(dg, orc, i):
     assert np.all(np.isfinite(P.bits_to_f64(got)))
     rows = P.sample_rows(case.M, 24, seed=i)
     ref = orc.gemm_dense(case.a, case.sa, case.b, case.sb, rows=rows)
-    P.assert_close(got[rows], ref.bits, ref.mag, f"sweep {i} {case.M}x{case.N}x{case.K}")
+    P.check(got[rows], ref, f"sweep {i} {case.M}x{case.N}x{case.K}")
 
 
 def test_prefill_full_size_sampled(dg, orc):
@@ -123,7 +123,7 @@ def test_prefill_full_size_sampled(dg, orc):
     assert not np.any(got == P.SENTINEL)
     rows = P.sample_rows(case.M, 40, seed=55)
     ref = orc.gemm_dense(case.a, case.sa, case.b, case.sb, rows=rows)
-    P.assert_close(got[rows], ref.bits, ref.mag, "prefill")
+    P.check(got[rows], ref, "prefill")
 
 
 # ---- contiguous ----------------------------------------------------------------------------
@@ -135,7 +135,7 @@ def _contig_check(dg, orc, case, rows=None, what="contiguous"):
     assert np.all(got[pad] == P.SENTINEL), "a padding row was written"
     ref = orc.gemm_contiguous(case.a, case.sa, case.b, case.sb, case.m_indices, rows=rows)
     check = ~pad if rows is None else np.isin(np.arange(case.M_total), rows) & ~pad
-    P.assert_close(got[check], ref.bits[check], ref.mag[check], what)
+    P.check(got, ref, what, sel=check)
     assert dg.poll_device_error() == 0
     return got
 
@@ -159,9 +159,7 @@ def test_contiguous_all_padding_tile(dg, orc):
 
 def test_contiguous_config_full_size_sampled(dg, orc):
     case = workloads.contiguous_case()
-    valid = np.nonzero(case.m_indices >= 0)[0]
-    rng = np.random.default_rng(3)
-    rows = np.unique(np.concatenate([valid[:3], valid[-3:], rng.choice(valid, 40, replace=False)]))
+    rows = P.sample_valid_rows(case.m_indices >= 0, 40, seed=3)
     _contig_check(dg, orc, case, rows=rows, what="contiguous config")
 
 
@@ -178,6 +176,29 @@ def test_contiguous_nan_in_padding_rows_isolated(dg, orc):
     assert np.array_equal(clean[~pad], dirty[~pad])
     assert np.all(np.isfinite(P.bits_to_f64(dirty[~pad])))
     assert np.all(dirty[pad] == P.SENTINEL)
+
+
+def test_contiguous_index_below_minus_one_reports_layout_error(dg, orc):
+    """An expert index below -1 (only -1 marks padding) breaks the layout contract: the device
+    sets DG_ERR_LAYOUT, the row is not written, and the other rows are still correct -- also
+    when a whole tile holds such indices."""
+    case = workloads.contiguous(G=2, N=128, K=256, seed=16, counts=[128, 100])
+    case.m_indices = case.m_indices.copy()
+    case.m_indices[5] = -2
+    case.m_indices[200] = np.iinfo(np.int32).min
+    got = P.out_bits(P.run_contiguous(dg, case))
+    assert dg.poll_device_error() == dg.DG_ERR_LAYOUT
+    assert np.all(got[5] == P.SENTINEL) and np.all(got[200] == P.SENTINEL)
+    ok = case.m_indices >= 0
+    ref = orc.gemm_contiguous(case.a, case.sa, case.b, case.sb, np.where(ok, case.m_indices, -1))
+    P.check(got, ref, "index below -1", sel=ok)
+    assert np.all(got[~ok] == P.SENTINEL)
+    # a tile whose every index is -2 is skipped and still reported
+    case2 = workloads.contiguous(G=1, N=64, K=128, seed=17, counts=[128])
+    case2.m_indices = np.full_like(case2.m_indices, -2)
+    got2 = P.out_bits(P.run_contiguous(dg, case2))
+    assert dg.poll_device_error() == dg.DG_ERR_LAYOUT
+    assert np.all(got2 == P.SENTINEL)
 
 
 def test_contiguous_mixed_expert_tile_reports_layout_error(dg):
@@ -206,7 +227,7 @@ def _masked_check(dg, orc, case, rows=None, what="masked"):
         sel = np.zeros(case.G * case.M_max, bool)
         sel[rows] = True
         valid &= sel.reshape(case.G, case.M_max)
-    P.assert_close(got[valid], ref.bits[valid], ref.mag[valid], what)
+    P.check(got, ref, what, sel=valid)
     assert dg.poll_device_error() == 0
     return got
 
@@ -220,6 +241,21 @@ def test_masked_small_edge_counts(dg, orc):
 def test_masked_all_empty(dg, orc):
     case = workloads.masked(G=3, M_max=128, N=64, K=128, seed=22, masked_m=[0, 0, 0])
     _masked_check(dg, orc, case)
+
+
+@pytest.mark.parametrize("family", [1, 2])
+def test_masked_largest_group_count(dg, orc, family):
+    """G = 1024, the largest group count the masked call takes: the tile prefix over groups
+    fills its last slot.  Most groups are empty; the last group and a few others hold rows."""
+    G = 1024
+    mm = np.zeros(G, np.int64)
+    mm[[0, 3, 511, 1000, G - 1]] = [128, 1, 77, 128, 100]
+    case = workloads.masked(G=G, M_max=128, N=256, K=128, seed=26, masked_m=mm)
+    dg.set_kernel_family(family)
+    try:
+        _masked_check(dg, orc, case, what=f"masked G=1024 family {family}")
+    finally:
+        dg.set_kernel_family(0)
 
 
 def test_masked_m_max_not_multiple_of_128(dg, orc):
@@ -287,5 +323,5 @@ def test_tensor_map_cache_hits_and_matches_uncached(dg, orc):
         dg.set_tensor_map_cache(prev)
     assert np.array_equal(uncached, first)
     ref = orc.gemm_dense(case.a, case.sa, case.b, case.sb)
-    P.assert_close(first, ref.bits, ref.mag, "cached maps")
+    P.check(first, ref, "cached maps")
     assert dg.poll_device_error() == 0

@@ -125,3 +125,45 @@ def test_quantise_matches_numpy_torch_composition():
     q, sa = oracle.quantize_1x128(bits)
     assert np.array_equal(sa, s)
     assert np.array_equal(q, ref_q)
+
+
+def test_quantise_departs_from_the_division_form_only_next_to_midpoints():
+    """Bounds the oracle's quantiser against the plain definition of the quantisation,
+    code = e4m3(x / scale) with scale = amax / 448 -- the form the GEMM harness uses for its
+    synthetic inputs, here evaluated as one fp32 division and cast by torch's independent
+    float8_e4m3fn conversion.  The oracle multiplies by the fp32 factor 448 / amax instead.  Both
+    quotients lie within 2^-24 relative (one fp32 rounding each, plus the rounding of the factor
+    or of the scale) of the exact x / scale, so where the two codes differ an E4M3 rounding
+    midpoint must lie within a few 2^-24 of it, and the codes must be neighbours (same sign,
+    magnitudes one code apart).  Everywhere else the codes are equal."""
+    rng = np.random.default_rng(14)
+    M, K = 2048, 1024
+    x = rng.normal(0, 1, (M, K)).astype(np.float32)
+    x[rng.random((M, K)) < 0.01] *= 50.0
+    x[: M // 4] = rng.uniform(-3.0, 3.0, (M // 4, K)).astype(np.float32)
+    x[M // 4: M // 2] *= np.float32(1e-3)          # tiles reaching the subnormal codes
+    bits = _bf16_bits(x)
+    xf = _bits_to_f32(bits)
+    q, sa = oracle.quantize_1x128(bits)
+    s_full = np.repeat(sa, 128, axis=1)
+    div32 = (xf / s_full).astype(np.float32)
+    q_div = torch.from_numpy(np.clip(div32, -448, 448)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    # the exact quotient (fp64 holds x / scale of two fp32 numbers to 2^-53) and its distance to
+    # the nearest rounding midpoint of the E4M3 grid, relative to the quotient
+    v = np.abs(xf.astype(np.float64) / s_full.astype(np.float64))
+    grid = np.array([oracle.e4m3_decode(c) for c in range(0x7F)])      # +0 .. 448, ascending
+    mids = (grid[:-1] + grid[1:]) / 2
+    pos = np.clip(np.searchsorted(mids, v), 1, mids.size - 1)
+    near = np.minimum(np.abs(v - mids[pos - 1]), np.abs(v - mids[pos]))
+    rel = np.where(v > 0, near / np.maximum(v, 1e-300), np.inf)
+    differ = q != q_div
+    n_near = int(np.count_nonzero(rel < 2.0 ** -21))
+    assert n_near > 0, "the sample reached no midpoint: the bound below would be untested"
+    assert np.all(rel[differ] < 2.0 ** -21), "codes differ away from a midpoint"
+    same_sign = (q[differ] & 0x80) == (q_div[differ] & 0x80)
+    step = np.abs((q[differ] & 0x7F).astype(int) - (q_div[differ] & 0x7F).astype(int))
+    assert np.all(same_sign) and np.all(step == 1), "differing codes are not neighbours"
+    assert np.count_nonzero(differ) <= n_near
+    # the scales are the plain definition amax / 448 (floored), bit for bit
+    amax = np.maximum(np.abs(xf.reshape(M, K // 128, 128)).max(axis=2), np.float32(1e-4))
+    assert np.array_equal(sa, (amax / np.float32(448.0)).astype(np.float32))

@@ -191,6 +191,117 @@ def with_fp4_b(case, seed: int, b_std: float = 0.02):
     return dataclasses.replace(case, b=b, sb=sb)
 
 
+# ---- edge-value inputs ---------------------------------------------------------------------
+# Codes and scales drawn directly (no fp32 source, no quantisation) so that the inputs reach the
+# values two-level accumulation exists for: products that cancel inside one 128-wide K slice,
+# slices whose sums pass fp32's exact-integer range, every finite code including subnormals,
+# and block scales whose products span 2^-60 .. 2^60.
+
+E4M3_POS_MAX = 0x7E          # +448
+E4M3_NAN = 0x7F              # the two NaN codes are 0x7F and 0xFF
+E4M3_FINITE = np.array([c for c in range(256) if (c & 0x7F) != E4M3_NAN], np.uint8)  # 254 codes
+E2M1_POS_MAX = 0x7           # +6 (sign in bit 3)
+EDGE_PATTERNS = ("cancel", "cancel_residual", "pm_max", "all_codes")
+
+
+def pack_e2m1(nibbles: np.ndarray) -> np.ndarray:
+    """E2M1 codes [..., K] (one per uint8, low 4 bits) -> packed bytes [..., K/2], element 2j in
+    the low nibble of byte j."""
+    n = np.asarray(nibbles, np.uint8) & 0xF
+    return (n[..., 0::2] | (n[..., 1::2] << 4)).astype(np.uint8)
+
+
+def _signed(rng, mag_codes: np.ndarray, sign_bit: int) -> np.ndarray:
+    signs = rng.integers(0, 2, mag_codes.shape).astype(np.uint8) * np.uint8(sign_bit)
+    return (mag_codes.astype(np.uint8) | signs).astype(np.uint8)
+
+
+def _edge_codes(pattern: str, rows: int, K: int, rng, fp4: bool, cancel_k, big_sign, second_sign):
+    """Codes [rows, K] of one operand.  fp4: E2M1 codes (one per byte), else E4M3 codes.
+    cancel_k[kb] = (k0, k1): the two positions of K block kb that carry the largest magnitude;
+    big_sign [rows] (0/1) is the sign of the first, second_sign [rows] that of the second."""
+    sign_bit = 0x8 if fp4 else 0x80
+    big = E2M1_POS_MAX if fp4 else E4M3_POS_MAX
+    if pattern == "all_codes":
+        pool = np.arange(16, dtype=np.uint8) if fp4 else E4M3_FINITE
+        return pool[rng.integers(0, pool.size, (rows, K))]
+    if pattern == "pm_max":
+        return _signed(rng, np.full((rows, K), big, np.uint8), sign_bit)
+    # cancel / cancel_residual: small magnitudes everywhere (E4M3: subnormals 2^-9 .. 7 * 2^-9
+    # and the smallest normals; E2M1: 0.5 .. 1.5), the largest magnitude at k0 and k1
+    lo, hi = (1, 3) if fp4 else (1, 12)
+    c = _signed(rng, rng.integers(lo, hi + 1, (rows, K)).astype(np.uint8), sign_bit)
+    for kb, (k0, k1) in enumerate(cancel_k):
+        c[:, k0] = big | (big_sign * sign_bit)
+        c[:, k1] = big | (second_sign * sign_bit)
+    return c.astype(np.uint8)
+
+
+def edge_dense(pattern: str, M: int, N: int, K: int, seed: int, fp4: bool = False,
+               scale_exp: int = 30) -> Dense:
+    """A Dense case with edge-value codes (see EDGE_PATTERNS):
+      cancel          per K block, positions k0 != k1 hold +-448 in A (the same sign at both)
+                      and +-448 / -+448 in B (opposite signs), so the two largest products of
+                      every slice cancel exactly; every other product is tiny (subnormal
+                      codes), so the slice's sum is far below its magnitude;
+      cancel_residual the same with B's second large code one step smaller (E4M3 416, E2M1
+                      4): the slice keeps a residual (448 * 32, or 448 * 2) next to the tiny
+                      products;
+      pm_max          every code +-448 (E2M1: +-6): a slice of equal signs sums to 128 * 448^2,
+                      past fp32's exact-integer range 2^24;
+      all_codes       codes uniform over the 254 finite E4M3 codes (E2M1: all 16 codes).
+    Scales are powers of two 2^U{-scale_exp .. scale_exp} per 1x128 A tile and per 128x128 B
+    block, so sa * sb spans 2^-60 .. 2^60 at the default.  fp4: B is a packed E2M1 operand
+    [N, K/2] (A stays E4M3).  Draw order: positions, signs, A, B, sa, sb."""
+    assert pattern in EDGE_PATTERNS and K % BLOCK == 0
+    rng = np.random.default_rng(seed)
+    Kb, Nb = K // BLOCK, -(-N // BLOCK)
+    cancel_k = []
+    for kb in range(Kb):
+        k0, k1 = rng.choice(BLOCK, 2, replace=False)
+        cancel_k.append((kb * BLOCK + int(k0), kb * BLOCK + int(k1)))
+    sa_sign = rng.integers(0, 2, (M,)).astype(np.uint8)
+    sb_sign = rng.integers(0, 2, (N,)).astype(np.uint8)
+    a = _edge_codes(pattern, M, K, rng, False, cancel_k, sa_sign, sa_sign)
+    b = _edge_codes(pattern, N, K, rng, fp4, cancel_k, sb_sign, 1 - sb_sign)
+    if pattern == "cancel_residual":
+        smaller = 0x6 if fp4 else 0x7D       # E2M1 4 (the step below 6), E4M3 416
+        for k0, k1 in cancel_k:
+            b[:, k1] = (b[:, k1] & (0x8 if fp4 else 0x80)) | smaller
+    sa = np.ldexp(1.0, rng.integers(-scale_exp, scale_exp + 1, (M, Kb))).astype(np.float32)
+    sb = np.ldexp(1.0, rng.integers(-scale_exp, scale_exp + 1, (Nb, Kb))).astype(np.float32)
+    if fp4:
+        b = pack_e2m1(b)
+    return Dense(M, N, K, a, sa, b, sb)
+
+
+def edge_contiguous(pattern: str, N: int, K: int, seed: int, rows: int = 200, fp4: bool = False) -> Contiguous:
+    """One expert segment (expert 1 of G = 2; expert 0 has no rows) of ``rows`` edge-value
+    rows, padded to a multiple of 128 with -1 rows."""
+    d = edge_dense(pattern, rows, N, K, seed, fp4=fp4)
+    M_total = -(-rows // BLOCK) * BLOCK
+    a = np.zeros((M_total, K), np.uint8)
+    sa = np.ones((M_total, K // BLOCK), np.float32)
+    a[:rows], sa[:rows] = d.a, d.sa
+    mi = np.full(M_total, -1, np.int32)
+    mi[:rows] = 1
+    b = np.stack([np.zeros_like(d.b), d.b])
+    sb = np.stack([np.ones_like(d.sb), d.sb])
+    return Contiguous(2, N, K, np.array([0, rows], np.int64), mi, a, sa, b, sb)
+
+
+def edge_masked(pattern: str, N: int, K: int, seed: int, rows: int = 200, M_max: int = 256,
+                fp4: bool = False) -> Masked:
+    """One masked group (group 1 of G = 2 holds ``rows`` valid edge-value rows; group 0 has
+    none); rows past masked_m are filled too."""
+    d = edge_dense(pattern, M_max, N, K, seed, fp4=fp4)
+    a = np.stack([np.zeros_like(d.a), d.a])
+    sa = np.stack([np.ones_like(d.sa), d.sa])
+    b = np.stack([np.zeros_like(d.b), d.b])
+    sb = np.stack([np.ones_like(d.sb), d.sb])
+    return Masked(2, M_max, N, K, rows, np.array([0, rows], np.int32), a, sa, b, sb)
+
+
 # ---- the named workloads ----------------------------------------------------------------
 
 SMALL_DENSE = dict(M=128, N=256, K=512)
