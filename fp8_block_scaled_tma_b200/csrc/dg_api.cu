@@ -281,11 +281,14 @@ constexpr int kPairSfaRingBytes = dg::kSfaSlots * dg::kKbPerStage * dg::kBlockM 
 // Tile heuristic of the pair kernel: 256-row pair tiles, waves over SM pairs.
 // Time model shared by the tile choosers.  A persistent CTA (or CTA pair) walks its tiles one
 // after another, so the time is (tiles per CTA, rounded up) x (time of one tile).  Measured on
-// B200 (dense 4096-row shapes, every BN from 128 to 256, both kernel families), one K block of
-// one 128-row tile costs about kTileFixed + BN column-units: a fixed part (the MMA-commit ->
-// promotion -> buffer-release round trip) plus a part proportional to the tile width (MMA,
-// tensor-memory reads and FFMA promotion).  Columns computed past N are wasted work.
-constexpr double kTileFixed = 190.0;
+// B200 (dense 4096-row shapes, BN from 160 to 256, both kernel families), one K block of one
+// tile costs about kTileFixed + BN column-units: a fixed part (the MMA-commit -> promotion ->
+// buffer-release round trip, ~600-750 cycles) plus ~1.5-2 cycles per column (MMA, tensor-memory
+// reads and FFMA promotion); the CTA-pair kernel is nearly flat in BN.  So whole waves decide,
+// and among equal wave counts the narrower tile wins.  Columns computed past N are wasted work.
+// (An earlier fit with a fixed part of 190 units picked BN = 224 for 8192 x 7168 x 18432, 14
+// waves of pair tiles, where BN = 256 runs 13 waves and measured 3 % faster.)
+constexpr double kTileFixed = 400.0;
 // Dense problems use CTA pairs only for long K: measured on B200, the pair kernel is ahead by a
 // few percent at K = 16384 and level with or behind the one-CTA kernel at K <= 7168, where its
 // longer per-tile start-up weighs more.

@@ -263,12 +263,14 @@ __device__ __forceinline__ bool promote_kb(float (&acc)[NCOLS], float sa, float 
         release();  // the whole partial is in registers: free the buffer before the arithmetic
     const float scale_lo = sa * sb_lo;
     const float scale_hi = sa * sb_hi;
+    // two columns per packed FMA (the promotion's FMAs sit between the two TMEM reads of a
+    // wide tile, on the path that recycles the buffer: half the instructions shortens it)
 #pragma unroll
     for (int g16 = 0; g16 < P1 / 16; ++g16) {
-        const float f = (16 * g16 >= split) ? scale_hi : scale_lo;
+        const uint64_t ff = ptx::pack_f32x2((16 * g16 >= split) ? scale_hi : scale_lo);
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-            acc[16 * g16 + e] = fmaf(__uint_as_float(pr[16 * g16 + e]), f, acc[16 * g16 + e]);
+        for (int e = 0; e < 16; e += 2)
+            ptx::ffma2(acc[16 * g16 + e], acc[16 * g16 + e + 1], pr[16 * g16 + e], pr[16 * g16 + e + 1], ff);
     }
     if (P2 > 0) {
         // second part reuses the same registers
@@ -277,10 +279,11 @@ __device__ __forceinline__ bool promote_kb(float (&acc)[NCOLS], float sa, float 
         release();
 #pragma unroll
         for (int g16 = 0; g16 < P2 / 16; ++g16) {
-            const float f = (P1 + 16 * g16 >= split) ? scale_hi : scale_lo;
+            const uint64_t ff = ptx::pack_f32x2((P1 + 16 * g16 >= split) ? scale_hi : scale_lo);
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-                acc[P1 + 16 * g16 + e] = fmaf(__uint_as_float(pr[16 * g16 + e]), f, acc[P1 + 16 * g16 + e]);
+            for (int e = 0; e < 16; e += 2)
+                ptx::ffma2(acc[P1 + 16 * g16 + e], acc[P1 + 16 * g16 + e + 1], pr[16 * g16 + e],
+                           pr[16 * g16 + e + 1], ff);
         }
     }
     return true;

@@ -431,6 +431,30 @@ __device__ __forceinline__ void mma_commit_pair_local(uint32_t bar)
         : "memory");
 }
 
+// ---- packed fp32 arithmetic ----------------------------------------------------------------
+
+// {f, f} in one 64-bit register: the second operand of ffma2 when both lanes scale alike.
+__device__ __forceinline__ uint64_t pack_f32x2(float f)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(f));
+    return r;
+}
+
+// acc0 += p0 * f, acc1 += p1 * f as one two-lane fp32 FMA (fma.rn.f32x2, sm_100): each lane is
+// an ordinary fp32 fused multiply-add rounded to nearest even, bit for bit what fmaf gives, in
+// half the issued instructions.  p0 / p1 are fp32 bit patterns; ff = pack_f32x2(f).
+__device__ __forceinline__ void ffma2(float &acc0, float &acc1, uint32_t p0, uint32_t p1, uint64_t ff)
+{
+    asm("{\n\t.reg .b64 a, c;\n\t"
+        "mov.b64 a, {%2, %3};\n\t"
+        "mov.b64 c, {%0, %1};\n\t"
+        "fma.rn.f32x2 c, a, %4, c;\n\t"
+        "mov.b64 {%0, %1}, c;\n\t}"
+        : "+f"(acc0), "+f"(acc1)
+        : "r"(p0), "r"(p1), "l"(ff));
+}
+
 // ---- misc -----------------------------------------------------------------------------------
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)

@@ -58,23 +58,31 @@ def compare(got_bits: np.ndarray, ref_bits: np.ndarray, mag: np.ndarray, acc=Non
                 first_bad=None if not bad.any() else tuple(int(i) for i in np.argwhere(bad)[0]))
 
 
-def assert_close(got_bits, ref_bits, mag, what: str, acc) -> dict:
+def assert_close(got_bits, ref_bits, mag, what: str, acc, matrix: bool = True) -> dict:
     """The parity bar: every element within tolerance, the matrix difference within DIFF_MAX,
     and the error beyond one bf16 rounding within EXCESS_MAX of the magnitude.  ``acc`` is the
-    oracle's unrounded fp64 result for the same entries (required)."""
+    oracle's unrounded fp64 result for the same entries (required).
+
+    matrix=False drops the matrix criterion, for inputs built so that every exact result is the
+    residue of a catastrophic cancellation (|Dref| ~ 1e-8 of sum |ab|).  There the matrix
+    difference compares errors of fp32 accumulation (~2^-24 of the cancelled magnitude, which
+    the two-level method accepts inside each 128-wide slice) with the tiny residues themselves,
+    and no fp32-accumulating implementation meets it; the element and excess bounds, which are
+    relative to the magnitude, still apply."""
     r = compare(got_bits, ref_bits, mag, acc)
     assert r["n_bad"] == 0, f"{what}: {r['n_bad']}/{r['n']} elements out of tolerance, first at {r['first_bad']}: {r}"
-    assert r["diff"] <= DIFF_MAX, f"{what}: matrix diff {r['diff']} > {DIFF_MAX}"
+    if matrix:
+        assert r["diff"] <= DIFF_MAX, f"{what}: matrix diff {r['diff']} > {DIFF_MAX}"
     assert r["excess"] < EXCESS_MAX, f"{what}: error beyond one bf16 rounding {r['excess']} >= {EXCESS_MAX}"
     return r
 
 
-def check(got_bits, ref, what: str, sel=None) -> dict:
+def check(got_bits, ref, what: str, sel=None, matrix: bool = True) -> dict:
     """assert_close against an oracle Result, optionally on a selection ``sel`` (an index or
     mask applied alike to the GPU bits and to the oracle's arrays)."""
     if sel is None:
-        return assert_close(got_bits, ref.bits, ref.mag, what, ref.acc)
-    return assert_close(got_bits[sel], ref.bits[sel], ref.mag[sel], what, ref.acc[sel])
+        return assert_close(got_bits, ref.bits, ref.mag, what, ref.acc, matrix)
+    return assert_close(got_bits[sel], ref.bits[sel], ref.mag[sel], what, ref.acc[sel], matrix)
 
 
 def to_dev_u8(x: np.ndarray) -> torch.Tensor:
