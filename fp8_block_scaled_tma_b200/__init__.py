@@ -180,7 +180,19 @@ def get_num_sms() -> int:
 
 
 def get_workspace_size(kind: int, M: int, N: int, K: int, G: int = 1) -> int:
+    """Bytes of workspace the stream-K kernel (kernel family 5, dense M <= 64) needs for this
+    call (0: it does not apply).  Allocate it zero-filled, e.g. with workspace_for, and keep one
+    per stream.  Automatic mode never needs one."""
     return int(lib.dg_get_workspace_size(kind, M, N, K, G))
+
+
+def workspace_for(M: int, N: int, K: int, device=None):
+    """A zero-filled workspace for dense calls of this size on the current device (None when
+    the call uses none)."""
+    n = get_workspace_size(0, M, N, K)
+    if n == 0:
+        return None
+    return torch.zeros(n, dtype=torch.uint8, device=device if device is not None else "cuda")
 
 
 def poll_device_error(stream=None) -> int:
@@ -210,8 +222,9 @@ FAMILY_AUTO, FAMILY_ONE_CTA, FAMILY_PAIR, FAMILY_SPLIT_K = 0, 1, 2, 3
 
 def set_kernel_family(family: int) -> int:
     """0 automatic, 1 one-CTA kernels, 2 CTA-pair kernels where the layout allows, 3 split-K
-    cluster kernel for dense calls, 4 swapped-operand kernel for dense calls with M <= 128.
-    Returns the previous value."""
+    cluster kernel for dense calls, 4 swapped-operand kernel for dense calls with M <= 128,
+    5 stream-K swapped-operand kernel for dense calls with M <= 64 (needs the workspace of
+    get_workspace_size).  Returns the previous value."""
     r = lib.dg_set_kernel_family(int(family))
     if r < 0:
         raise DGError(r, "dg_set_kernel_family")

@@ -17,6 +17,7 @@
 #include "dg_quant_kernel.cuh"
 #include "dg_splitk_kernel.cuh"
 #include "dg_swap_kernel.cuh"
+#include "dg_swap_sk_kernel.cuh"
 
 namespace {
 
@@ -54,8 +55,9 @@ KernelSmem g_smem[kMaxDevices][3][8];       // 1-CTA kernels, per device / layou
 KernelSmem g_smem_pair[kMaxDevices][3][8];  // CTA-pair kernels
 KernelSmem g_smem_split[kMaxDevices][8];    // split-K kernels, per BN
 KernelSmem g_smem_swap[kMaxDevices][6];     // swapped-operand kernels, per (TN, R)
+KernelSmem g_smem_swap_sk[kMaxDevices][2];  // stream-K swapped-operand kernels, per TN (32, 64)
 // 0 auto, 1 one-CTA kernels, 2 CTA pairs where possible, 3 split-K (dense), 4 swapped operands
-// (dense, M <= 128)
+// (dense, M <= 128), 5 stream-K swapped operands (dense, M <= 64, needs the caller's workspace)
 int g_family = 0;
 int g_num_sms_cap = 0;
 unsigned long long g_timeout_ns = kDefaultTimeoutNs;
@@ -476,6 +478,8 @@ struct LaunchArgs {
     int expected_m;
     void *stream;
     int b_fp4 = 0;  // B holds packed E2M1 (two per byte) instead of E4M3 codes
+    void *ws = nullptr;      // caller's workspace (dense calls; may be null)
+    size_t ws_bytes = 0;
 };
 
 int launch_splitk(const LaunchArgs &args, int dev, DeviceInfo *info, int bn, int S,
@@ -945,6 +949,157 @@ int launch_swap(const LaunchArgs &args, int dev, DeviceInfo *info, int R, int S,
     return DG_OK;
 }
 
+// ---- stream-K swapped-operand kernel (dense, M <= 64, caller's workspace) --------------------
+
+template <int TN>
+void *swap_sk_kernel_ptr()
+{
+    return reinterpret_cast<void *>(&dg::dg_gemm_swap_sk_kernel<TN>);
+}
+
+void *pick_swap_sk_kernel(int tn)
+{
+    return tn == 32 ? swap_sk_kernel_ptr<32>() : tn == 64 ? swap_sk_kernel_ptr<64>() : nullptr;
+}
+
+// The stream-K plan of a dense call: P CTAs (one per SM), U = tiles x K/128 units, at most H
+// units per CTA.  Returns false where the kernel does not apply: more than 64 tokens, fewer
+// units than SMs, more tiles than SMs (a CTA's range would span three tiles), or an A-scale box
+// taller than TMA allows.
+struct SkPlan {
+    int tn = 0, P = 0, n_tiles = 0, H = 0;
+    size_t part_bytes = 0, count_bytes = 0;
+    size_t total() const { return part_bytes + count_bytes; }
+};
+
+bool plan_swap_sk(int M, int N, int K, int sms, SkPlan &pl)
+{
+    if (M < 1 || M > 64 || sms < 1)
+        return false;
+    const int num_kb = K / dg::kBlockK;
+    pl.tn = swap_token_tile(M);
+    pl.n_tiles = (N + dg::kBlockM - 1) / dg::kBlockM;
+    pl.P = sms;
+    const long long U = static_cast<long long>(pl.n_tiles) * num_kb;
+    if (pl.n_tiles > pl.P || U < pl.P)
+        return false;
+    pl.H = static_cast<int>((U + pl.P - 1) / pl.P);
+    if (pl.H > 256 || pl.H > num_kb)
+        return false;
+    pl.part_bytes = static_cast<size_t>(pl.P) * 2 * pl.tn * dg::kBlockM * 4;
+    pl.count_bytes = (static_cast<size_t>(pl.n_tiles) * 4 + 255) / 256 * 256;
+    return true;
+}
+
+int launch_swap_sk(const LaunchArgs &args, int dev, DeviceInfo *info, const SkPlan &pl, float *ws,
+                   int *ws_count, int stages_override, unsigned long long timeout)
+{
+    const int M = args.M, N = args.N, K = args.K;
+    const int num_kb = K / dg::kBlockK;
+    const int num_nb = (N + dg::kBlockK - 1) / dg::kBlockK;
+    void *fn = pick_swap_sk_kernel(pl.tn);
+    if (fn == nullptr)
+        return DG_ERR_INVALID_ARG;
+    const int idx = pl.tn == 32 ? 0 : 1;
+    const int sbytes = swap_stage_bytes(pl.tn, 1);
+    const int scale_bytes = 2 * pl.H * pl.tn * 4;
+    int stages = 0, dyn_smem = 0;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        KernelSmem &ks = g_smem_swap_sk[dev][idx];
+        if (ks.static_bytes < 0) {
+            cudaFuncAttributes fa;
+            cudaError_t e = cudaFuncGetAttributes(&fa, fn);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                return DG_ERR_CUDA;
+            }
+            ks.static_bytes = static_cast<int>(fa.sharedSizeBytes);
+        }
+        const int dyn_cap = info->smem_optin - ks.static_bytes;
+        stages = std::min(dg::kMaxStages, (dyn_cap - 1024 - scale_bytes) / sbytes);
+        if (stages_override > 0)
+            stages = std::min(stages, stages_override);
+        if (stages < 2)
+            return DG_ERR_UNSUPPORTED;
+        dyn_smem = stages * sbytes + scale_bytes + 1024;
+        dyn_smem = std::min(std::max(dyn_smem, kMinDynSmem), dyn_cap);
+        if (ks.limit_set < dyn_smem) {
+            cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                return DG_ERR_CUDA;
+            }
+            ks.limit_set = dyn_smem;
+        }
+    }
+    const int sfa_ld = align4(M);
+    CUtensorMap map_a, map_b, map_sa;
+    if (make_map_kblocks(&map_a, const_cast<void *>(args.a), K, M, 1, pl.tn, dg::kSwapKbPerStage) != DG_OK ||
+        make_map_kblocks(&map_b, const_cast<void *>(args.b), K, N, 1, dg::kBlockM, dg::kSwapKbPerStage,
+                         args.b_fp4 != 0) != DG_OK ||
+        make_map(&map_sa, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, const_cast<float *>(args.sfa), sfa_ld, num_kb, 1,
+                 static_cast<uint64_t>(sfa_ld) * 4, static_cast<uint64_t>(sfa_ld) * 4 * num_kb, pl.tn, pl.H,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) != DG_OK) {
+        if (debug_enabled())
+            std::fprintf(stderr, "[dg] cuTensorMapEncodeTiled failed (stream-K)\n");
+        return DG_ERR_CUDA;
+    }
+    Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.G = 1;
+    p.num_kb = num_kb;
+    p.num_nb = num_nb;
+    p.m_tiles = pl.H;
+    p.n_tiles = pl.n_tiles;
+    p.num_tiles = pl.n_tiles;
+    p.stages = stages;
+    p.raster_m = pl.P;
+    p.sfa = args.sfa;
+    p.sfa_ld = sfa_ld;
+    p.sfb = args.sfb;
+    p.d = static_cast<__nv_bfloat16 *>(args.d);
+    p.err = info->err_ptr;
+    p.timeout_ns = timeout;
+    p.inject_stall = inject_stall_flag();
+    p.idesc_b = args.b_fp4 ? dg::ptx::kIdescBFormatE2M1 : 0u;
+    p.ws = ws;
+    p.ws_count = ws_count;
+
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(pl.P, 1, 1);
+    cfg.blockDim = dim3(dg::kNumThreads, 1, 1);
+    cfg.dynamicSmemBytes = dyn_smem;
+    cfg.stream = static_cast<cudaStream_t>(args.stream);
+    cudaLaunchAttribute attr[1];
+    cfg.attrs = attr;
+    cfg.numAttrs = add_pdl_attr(attr, 0);
+    void *kargs[] = {&map_a, &map_b, &map_sa, &p};
+    cudaError_t e = cudaLaunchKernelExC(&cfg, fn, kargs);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        if (debug_enabled())
+            std::fprintf(stderr, "[dg] stream-K launch failed: %s\n", cudaGetErrorString(e));
+        return DG_ERR_CUDA;
+    }
+    t_last.valid = true;
+    t_last.block_n = dg::kBlockM;
+    t_last.stages = stages;
+    t_last.grid = pl.P;
+    t_last.tiles = pl.n_tiles;
+    t_last.pair = 0;
+    t_last.splits = pl.H;
+    t_last.family = 5;
+    if (debug_enabled())
+        std::fprintf(stderr, "[dg] stream-K M=%d N=%d K=%d TN=%d P=%d H=%d stages=%d smem=%d\n", M, N, K,
+                     pl.tn, pl.P, pl.H, stages, dyn_smem);
+    return DG_OK;
+}
+
 int launch(const LaunchArgs &args)
 {
     int dev = 0;
@@ -982,6 +1137,20 @@ int launch(const LaunchArgs &args)
     // split-K on B200 (1-2 us on the 2112 / 4096 / 7168-wide decode shapes); with 65-128 tokens,
     // or when the tiles need two row blocks to fit in one wave, split-K and the one-CTA kernel
     // were level or faster.  (In auto mode a block_n override keeps the families it names.)
+    // Stream-K over every SM (dense M <= 64, family 5, the caller's workspace).  Automatic mode
+    // does not take it: on B200 it measured slower than the cluster kernels on every decode
+    // shape tried (64 x 7168 x 16384: 43.0 vs 36.9 us; 64 x 4096 x 7168: 26.1 vs 18.5 us), the
+    // partial round trip through L2 and the fix-up costing more than the SMs it adds.
+    if (args.layout == dg::kDense && pair_mode == 5) {
+        SkPlan pl;
+        if (!plan_swap_sk(M, N, K, sms, pl))
+            return DG_ERR_UNSUPPORTED;
+        if (args.ws == nullptr || args.ws_bytes < pl.total())
+            return DG_ERR_WORKSPACE;
+        float *ws = static_cast<float *>(args.ws);
+        int *cnt = reinterpret_cast<int *>(static_cast<char *>(args.ws) + pl.part_bytes);
+        return launch_swap_sk(args, dev, info, pl, ws, cnt, stages_override, timeout);
+    }
     const bool swap_auto = pair_mode == 0 && bn == 0 && M <= 64;
     if (args.layout == dg::kDense && M <= 128 && (pair_mode == 4 || swap_auto)) {
         int splits_override;
@@ -1323,7 +1492,7 @@ bool b_aligned(const void *b, int b_fp4)
 }
 
 int gemm_dense(const void *a, const float *sfa, const void *b, const float *sfb, void *d, int M,
-               int N, int K, void *stream, int b_fp4)
+               int N, int K, void *stream, int b_fp4, void *ws = nullptr, size_t ws_bytes = 0)
 {
     if (M < 0)
         return DG_ERR_INVALID_ARG;
@@ -1334,7 +1503,9 @@ int gemm_dense(const void *a, const float *sfa, const void *b, const float *sfb,
         return st;
     if (!b_aligned(b, b_fp4))
         return DG_ERR_INVALID_ARG;
-    LaunchArgs la{dg::kDense, a, sfa, b, sfb, d, nullptr, nullptr, M, N, K, 1, 0, stream, b_fp4};
+    if (ws != nullptr && (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+        return DG_ERR_INVALID_ARG;
+    LaunchArgs la{dg::kDense, a, sfa, b, sfb, d, nullptr, nullptr, M, N, K, 1, 0, stream, b_fp4, ws, ws_bytes};
     return launch(la);
 }
 
@@ -1385,9 +1556,7 @@ int dg_gemm_fp8_fp8_bf16_nt(const void *a, const float *sfa, const void *b, cons
                             void *d, int M, int N, int K, void *workspace, size_t workspace_bytes,
                             void *stream)
 {
-    (void)workspace;
-    (void)workspace_bytes;
-    return gemm_dense(a, sfa, b, sfb, d, M, N, K, stream, 0);
+    return gemm_dense(a, sfa, b, sfb, d, M, N, K, stream, 0, workspace, workspace_bytes);
 }
 
 int dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(const void *a, const float *sfa, const void *b,
@@ -1471,12 +1640,21 @@ int dg_get_tma_aligned_size(int x, int elem_bytes)
 
 size_t dg_get_workspace_size(int kind, int M, int N, int K, int G)
 {
-    (void)kind;
-    (void)M;
-    (void)N;
-    (void)K;
     (void)G;
-    return 0;
+    if (kind != 0 || N <= 0 || K <= 0 || K % dg::kBlockK != 0)
+        return 0;
+    int dev = 0;
+    DeviceInfo *info = nullptr;
+    if (device_setup(dev, info) != DG_OK)
+        return 0;
+    int sms = info->num_sms;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (g_num_sms_cap > 0 && g_num_sms_cap < sms)
+            sms = g_num_sms_cap;
+    }
+    SkPlan pl;
+    return plan_swap_sk(M, N, K, sms, pl) ? pl.total() : 0;
 }
 
 const char *dg_status_string(int status)
@@ -1584,7 +1762,7 @@ int dg_get_tensor_map_cache_stats(unsigned long long *hits, unsigned long long *
 
 int dg_set_kernel_family(int family)
 {
-    if (family < 0 || family > 4)
+    if (family < 0 || family > 5)
         return DG_ERR_INVALID_ARG;
     std::lock_guard<std::mutex> lock(g_mutex);
     int prev = g_family;

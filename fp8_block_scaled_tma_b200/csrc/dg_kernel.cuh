@@ -72,6 +72,8 @@ struct Params {
     int inject_stall;   // test hook: the MMA issuer first waits on a barrier nothing signals
     uint32_t idesc_b;   // B-format bits of the MMA instruction descriptor: 0 e4m3, or e2m1
                         // (FP4 B, staged by TMA in the padded 8-bit layout of kind::f8f6f4)
+    float *ws;          // stream-K kernel: the workspace's fp32 partial slots
+    int *ws_count;      // stream-K kernel: its per-tile arrival counters (zero between calls)
 };
 
 template <int BN>

@@ -53,8 +53,11 @@ typedef enum dg_status {
  *   a   e4m3 [M][K] row-major          sfa fp32 [K/128][align4(M)]  (MN-major)
  *   b   e4m3 [N][K] row-major          sfb fp32 [ceil(N/128)][K/128]
  *   d   bf16 [M][N] row-major (written: all M x N elements)
- * M >= 0 (M == 0 is a no-op).  workspace / workspace_bytes: pass NULL / 0 unless
- * dg_get_workspace_size(0, M, N, K, 1) > 0. */
+ * M >= 0 (M == 0 is a no-op).  workspace / workspace_bytes: used only by the stream-K kernel
+ * (kernel family 5, M <= 64; see dg_get_workspace_size), which needs at least
+ * dg_get_workspace_size(0, M, N, K, 1) bytes, 256-byte aligned and zero-filled before first use
+ * (DG_ERR_WORKSPACE otherwise); other calls accept NULL / 0.  A workspace that is not 256-byte
+ * aligned is DG_ERR_INVALID_ARG. */
 int dg_gemm_fp8_fp8_bf16_nt(const void *a, const float *sfa, const void *b, const float *sfb,
                             void *d, int M, int N, int K, void *workspace,
                             size_t workspace_bytes, void *stream);
@@ -172,8 +175,18 @@ int dg_get_num_sms(void);
  * a this is align4(M).  Returns DG_ERR_INVALID_ARG for x < 0 or elem_bytes <= 0. */
 int dg_get_tma_aligned_size(int x, int elem_bytes);
 
-/* Bytes of workspace a call of `kind` (0 dense, 1 contiguous, 2 masked) with these sizes
- * needs.  0 means workspace may be NULL. */
+/* Bytes of workspace a call of `kind` (0 dense, 1 contiguous, 2 masked) with these sizes can
+ * use on the current device; 0 means the call uses none.  Only the stream-K kernel (kernel
+ * family 5 of dg_set_kernel_family, dense calls with M <= 64) uses one: every SM takes an equal
+ * share of the K blocks, each writes its fp32 partial sums into the workspace, and the last
+ * contributor of an output tile adds them in K order (deterministic) and writes D.  Automatic
+ * mode never needs a workspace (it measured slower than the cluster kernels on B200, so it is
+ * opt-in), and a call outside family 5 ignores one.  Layout, owned by the caller:
+ * [SMs][2][TN][128] fp32 partial slots, then one int32 arrival counter per 128-row tile of B.
+ * Zero-fill it before its first use; every call leaves the counters at zero again, except one
+ * that reports DG_ERR_TIMEOUT (zero-fill it again then).  Calls that share a workspace must not
+ * overlap on the GPU (use one per stream).  The size depends on the SM budget
+ * (dg_set_num_sms). */
 size_t dg_get_workspace_size(int kind, int M, int N, int K, int G);
 
 /* Static, human-readable text for a dg_status value. */
@@ -216,7 +229,10 @@ int dg_set_config_override(int block_n, int num_stages, int splits);
  * swapped-operand kernel for dense calls with M <= 128 (B rows on the MMA's 128-row side, the
  * tokens on its N side, K split over a cluster as in 3; block_n 128 or 256 of
  * dg_set_config_override selects one or two 128-row blocks of B per tile), other calls run as
- * in automatic mode.  Automatic mode uses the swapped-operand kernel for dense M <= 64 with one
+ * in automatic mode; 5 = the stream-K swapped-operand kernel for dense calls with M <= 64 (see
+ * dg_get_workspace_size; DG_ERR_WORKSPACE when the call's workspace is missing or too small,
+ * DG_ERR_UNSUPPORTED for shapes it does not take: fewer K blocks x tiles than SMs, more tiles
+ * than SMs).  Automatic mode uses the swapped-operand kernel for dense M <= 64 with one
  * 128-row block of B per tile (when no block_n override is set), split-K for dense M <= 256 when
  * more than one split pays (else the one-CTA kernel), pairs for dense M > 256 with
  * K >= 96 * 128, and the one-CTA kernels otherwise (contiguous and masked included).  Results agree within the parity tolerance whichever
@@ -246,8 +262,9 @@ int dg_set_tensor_map_cache(int enable);
 int dg_get_tensor_map_cache_stats(unsigned long long *hits, unsigned long long *misses);
 
 /* Describes the most recent launch on this host thread: fills any non-NULL pointer with the
- * chosen block_n, pipeline stages, grid size (CTAs), output tile count, kernel family (1, 2 or
- * 3 as in dg_set_kernel_family) and K splits per tile.  Returns DG_OK, or DG_ERR_INVALID_ARG
+ * chosen block_n, pipeline stages, grid size (CTAs), output tile count, kernel family (1 to 5
+ * as in dg_set_kernel_family) and K splits per tile (for the stream-K kernel: the most K blocks
+ * one CTA takes).  Returns DG_OK, or DG_ERR_INVALID_ARG
  * when nothing was launched yet. */
 int dg_get_last_launch(int *block_n, int *num_stages, int *grid, int *num_tiles, int *family,
                        int *splits);

@@ -102,14 +102,14 @@ def out_bits(d: torch.Tensor) -> np.ndarray:
     return d.view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-def run_dense(dg, case, d=None) -> torch.Tensor:
+def run_dense(dg, case, d=None, workspace=None) -> torch.Tensor:
     a = to_dev_u8(case.a)
     b = to_dev_u8(case.b)
     sfa = dg.sfa_mn_major(to_dev_f32(case.sa))
     sfb = to_dev_f32(case.sb)
     if d is None:
         d = sentinel_out((case.M, case.N))
-    dg.dg_gemm_fp8_fp8_bf16_nt(a, sfa, b, sfb, d)
+    dg.dg_gemm_fp8_fp8_bf16_nt(a, sfa, b, sfb, d, workspace=workspace)
     torch.cuda.synchronize()
     return d
 

@@ -76,8 +76,10 @@ def test_config_override_validation(dg):
     assert dg.lib.dg_set_config_override(0, 0, 9) == dg.DG_ERR_INVALID_ARG
     assert dg.lib.dg_set_config_override(96, 4, 3) == dg.DG_OK
     assert dg.lib.dg_set_config_override(0, 0, 0) == dg.DG_OK
-    assert dg.lib.dg_set_kernel_family(5) == dg.DG_ERR_INVALID_ARG
-    assert dg.lib.dg_set_kernel_family(4) == 0 and dg.lib.dg_set_kernel_family(0) == 4
+    assert dg.lib.dg_set_kernel_family(6) == dg.DG_ERR_INVALID_ARG
+    assert dg.lib.dg_set_kernel_family(-1) == dg.DG_ERR_INVALID_ARG
+    assert dg.lib.dg_set_kernel_family(5) == 0 and dg.lib.dg_set_kernel_family(4) == 5
+    assert dg.lib.dg_set_kernel_family(0) == 4
     assert dg.lib.dg_set_fault_injection(2) == dg.DG_ERR_INVALID_ARG
     assert dg.lib.dg_set_fault_injection(0) == dg.DG_OK
     assert dg.lib.dg_set_kernel_family(0) == dg.DG_OK
@@ -194,3 +196,13 @@ def test_quantize_rejects_bad_arguments(dg):
     assert L.dg_quantize_fp8_1x128(FAKE + 4, FAKE, FAKE, 4, 128, None) == dg.DG_ERR_INVALID_ARG
     assert L.dg_quantize_fp8_1x128(None, FAKE, FAKE, 4, 128, None) == dg.DG_ERR_INVALID_ARG
     assert L.dg_quantize_fp8_1x128(None, None, None, 0, 128, None) == dg.DG_OK  # empty: no-op
+
+
+def test_workspace_size_without_a_device(dg):
+    """Without a usable device no call can use a workspace: the size is 0 and workspace_for
+    gives None (the GEMMs never require one)."""
+    if torch.cuda.is_available():
+        pytest.skip("checks the no-device answer")
+    assert dg.get_workspace_size(0, 64, 7168, 16384) == 0
+    assert dg.workspace_for(64, 7168, 16384) is None
+    assert dg.get_workspace_size(1, 64, 7168, 16384) == 0
