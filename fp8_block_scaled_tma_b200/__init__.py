@@ -51,6 +51,7 @@ def _load() -> ctypes.CDLL:
     lib.dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked.argtypes = [vp, fp, vp, fp, vp, ip, i, i, i, i,
                                                              i, vp, sz, vp]
     lib.dg_gemm_fp8_fp4_bf16_nt.argtypes = [vp, fp, vp, fp, vp, i, i, i, vp]
+    lib.dg_gemm_fp8_fp8_bf16_nt_noalloc.argtypes = [vp, fp, vp, fp, vp, i, i, i, vp]
     lib.dg_m_grouped_gemm_fp8_fp4_bf16_nt_contiguous.argtypes = [vp, fp, vp, fp, vp, ip, i, i, i,
                                                                  i, vp]
     lib.dg_m_grouped_gemm_fp8_fp4_bf16_nt_masked.argtypes = [vp, fp, vp, fp, vp, ip, i, i, i, i,
@@ -58,7 +59,7 @@ def _load() -> ctypes.CDLL:
     for name in ("dg_gemm_fp8_fp8_bf16_nt", "dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous",
                  "dg_m_grouped_gemm_fp8_fp8_bf16_nt_masked", "dg_gemm_fp8_fp4_bf16_nt",
                  "dg_m_grouped_gemm_fp8_fp4_bf16_nt_contiguous",
-                 "dg_m_grouped_gemm_fp8_fp4_bf16_nt_masked"):
+                 "dg_m_grouped_gemm_fp8_fp4_bf16_nt_masked", "dg_gemm_fp8_fp8_bf16_nt_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     lib.dg_set_num_sms.argtypes = [i]
     lib.dg_set_num_sms.restype = i
@@ -301,6 +302,23 @@ def dg_gemm_fp8_fp8_bf16_nt(a, sfa, b, sfb, d, workspace=None, stream=None) -> N
     _check(lib.dg_gemm_fp8_fp8_bf16_nt(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K,
                                        _ptr(workspace), ws, _stream(stream)),
            "dg_gemm_fp8_fp8_bf16_nt")
+
+
+def dg_gemm_fp8_fp8_bf16_nt_noalloc(a, sfa, b, sfb, d, stream=None) -> None:
+    """dg_gemm_fp8_fp8_bf16_nt for callers that cannot allocate device memory: the stream-K
+    kernel with its scratch in an array built into the library (dense, M <= 64; see dg.h)."""
+    _fp8(a, "a")
+    _fp8(b, "b")
+    M, K = a.shape
+    N = b.shape[0]
+    if b.shape[1] != K:
+        raise ValueError("a and b disagree on K")
+    _f32(sfa, "sfa", (K // BLOCK, get_tma_aligned_size(M, 4)))
+    _f32(sfb, "sfb", (-(-N // BLOCK), K // BLOCK))
+    _out(d, (M, N))
+    _check(lib.dg_gemm_fp8_fp8_bf16_nt_noalloc(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K,
+                                               _stream(stream)),
+           "dg_gemm_fp8_fp8_bf16_nt_noalloc")
 
 
 def quantize_fp8_1x128(x, q=None, sfa=None, stream=None):

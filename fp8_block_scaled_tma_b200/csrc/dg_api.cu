@@ -1548,6 +1548,32 @@ int gemm_masked(const void *a, const float *sfa, const void *b, const float *sfb
     return launch(la);
 }
 
+// ---- the dense GEMM without any allocation: the stream-K kernel with built-in scratch ----------
+
+// Scratch of dg_gemm_fp8_fp8_bf16_nt_noalloc: the stream-K kernel's partial slots and, after
+// them, its per-tile arrival counters.  A file-scope device array, so every GPU that loads the
+// library holds it until the process exits.  Host code may not use its name as an address: the
+// device address is looked up once per device (noalloc_scratch) and passed to the kernel.
+constexpr size_t kNoAllocScratchBytes = size_t(12) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+void *g_noalloc_ptr[kMaxDevices];  // device address of the array, per device (null: not looked up)
+
+// The array's device address on the current device `dev`, looked up on the first call there.
+int noalloc_scratch(int dev, unsigned char *&ptr)
+{
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return DG_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = p;
+    }
+    ptr = static_cast<unsigned char *>(g_noalloc_ptr[dev]);
+    return DG_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -1557,6 +1583,53 @@ int dg_gemm_fp8_fp8_bf16_nt(const void *a, const float *sfa, const void *b, cons
                             void *stream)
 {
     return gemm_dense(a, sfa, b, sfb, d, M, N, K, stream, 0, workspace, workspace_bytes);
+}
+
+int dg_gemm_fp8_fp8_bf16_nt_noalloc(const void *a, const float *sfa, const void *b, const float *sfb,
+                                    void *d, int M, int N, int K, void *stream)
+{
+    if (M < 0)
+        return DG_ERR_INVALID_ARG;
+    if (M == 0)
+        return (N > 0 && N % 8 == 0 && K > 0 && K % dg::kBlockK == 0) ? DG_OK : DG_ERR_INVALID_ARG;
+    int st = check_common(a, sfa, b, sfb, d, N, K);
+    if (st != DG_OK)
+        return st;
+    if (!b_aligned(b, 0))
+        return DG_ERR_INVALID_ARG;
+    int dev = 0;
+    DeviceInfo *info = nullptr;
+    st = device_setup(dev, info);
+    if (st != DG_OK)
+        return st;
+    int sms = info->num_sms;
+    int stages_override;
+    unsigned long long timeout;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (g_num_sms_cap > 0 && g_num_sms_cap < sms)
+            sms = g_num_sms_cap;
+        stages_override = g_override_stages;
+        timeout = g_timeout_ns;
+    }
+    SkPlan pl;
+    if (!plan_swap_sk(M, N, K, sms, pl))
+        return DG_ERR_UNSUPPORTED;
+    if (pl.total() > kNoAllocScratchBytes)
+        return DG_ERR_WORKSPACE;  // more scratch than the built-in array holds
+    unsigned char *scratch = nullptr;
+    st = noalloc_scratch(dev, scratch);
+    if (st != DG_OK)
+        return st;
+    // the tile counters start at zero whatever an earlier call left there
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(scratch + pl.part_bytes, 0, pl.count_bytes, s) != cudaSuccess) {
+        cudaGetLastError();
+        return DG_ERR_CUDA;
+    }
+    LaunchArgs la{dg::kDense, a, sfa, b, sfb, d, nullptr, nullptr, M, N, K, 1, 0, stream, 0};
+    return launch_swap_sk(la, dev, info, pl, reinterpret_cast<float *>(scratch),
+                          reinterpret_cast<int *>(scratch + pl.part_bytes), stages_override, timeout);
 }
 
 int dg_m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(const void *a, const float *sfa, const void *b,

@@ -62,6 +62,29 @@ int dg_gemm_fp8_fp8_bf16_nt(const void *a, const float *sfa, const void *b, cons
                             void *d, int M, int N, int K, void *workspace,
                             size_t workspace_bytes, void *stream);
 
+/* The dense GEMM of dg_gemm_fp8_fp8_bf16_nt for callers that cannot allocate device memory,
+ * allocating nothing itself.  (The DeepGEMM pages have no counterpart: this is a calling
+ * convention of this library.)  Some callers may not call cudaMalloc or any allocating routine
+ * during their work: a serving loop whose device memory is planned and reserved up front, an
+ * operator running inside another runtime that receives only its inputs and outputs, or code on
+ * a latency-critical thread, where cudaMalloc can synchronise the device.  They cannot provide
+ * the workspace the stream-K kernel needs (dg_get_workspace_size), so this entry runs that
+ * kernel -- every SM streams an equal share of the K blocks -- with its scratch in an array
+ * built into the library: a file-scope device array of 12 MiB that every GPU loading the
+ * library holds until the process exits.
+ *   Same arguments, layouts and results as dg_gemm_fp8_fp8_bf16_nt (without the workspace);
+ *   takes dense calls with 1 <= M <= 64 whose tiles of 128 rows of B x K/128 number at least the
+ *   SMs, and no more tiles than SMs (DG_ERR_UNSUPPORTED otherwise); DG_ERR_WORKSPACE when the
+ *   partial sums would not fit the 12 MiB (with the 148 SMs of a B200: 9.25 MiB at M <= 64).
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress, once
+ *   per device, with that device current); make that first call before any stream capture.
+ *   Each call clears the array's tile counters on `stream` before its kernel.  Every call on a
+ *   device shares the one array, which keeps the last call's contents: calls that overlap on the
+ *   GPU (other streams, other host threads) race and must be serialised by the caller.
+ *   M == 0 is a no-op. */
+int dg_gemm_fp8_fp8_bf16_nt_noalloc(const void *a, const float *sfa, const void *b, const float *sfb,
+                                    void *d, int M, int N, int K, void *stream);
+
 /* Contiguous-layout grouped GEMM for MoE, "m_grouped_gemm_fp8_fp8_bf16_nt_contiguous" of
  * "如何使用" (the token rows of several experts are concatenated along M).
  *   a          e4m3 [M_total][K]          sfa fp32 [K/128][M_total]
