@@ -64,7 +64,7 @@ SPEC_HBM_GBS = 8000.0     # B200 HBM3e bandwidth (data sheet)
 # figure only while the sources still have that fingerprint, and null once a kernel changed
 # since the counters were taken; --traffic-bytes overrides it.
 MEASURED_TRAFFIC = {
-    "dense 8192x7168x18432": (1097988096 + 113367808, "7735b50e38823d48"),   # CTA pair BN 256
+    "dense 8192x7168x18432": (1094379776 + 112736512, "358a90c0e22a9612"),   # CTA pair BN 256
     "dg_quantize_1x128_kernel 8192x7168": (117451520 + 9024512, None),
     "dg_swiglu_quantize_1x128_kernel 16384x4096": (134243072 + 7325696, None),
 }
