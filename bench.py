@@ -251,6 +251,81 @@ def measure_cublas_fp8(n: int = 8192, reps: int = 10):
         return None
 
 
+LIBRARY_STICK = "vLLM cutlass_scaled_mm: CUTLASS block-scaled FP8 GEMM (1x128 A scales, 128x128 B scales)"
+
+
+def library_stick(shapes, reps: int = 10) -> list:
+    """A measuring stick for the same computation from a library: vLLM's cutlass_scaled_mm with
+    DeepSeek-style block scales, on seeded inputs of each (M, N, K), timed beside this library's
+    dense GEMM on the same inputs (256 MiB L2 flush and a short sleep before every run, median
+    of `reps` event-timed runs after warm-up), with the largest difference between the two
+    outputs relative to |ours| + 1.  Runs in a child process (`--library-stick`) so that the
+    library's import cannot touch this process; never on the product path."""
+    import subprocess
+    arg = ";".join(f"{m},{n},{k}" for m, n, k in shapes)
+    try:
+        r = subprocess.run([sys.executable, os.path.abspath(__file__), "--library-stick", arg,
+                            "--steps", str(reps), "--warmup", "3"],
+                           capture_output=True, text=True, timeout=300)
+        lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+        if r.returncode != 0 or not lines:
+            tail = (r.stderr or r.stdout).strip().splitlines()[-1:] or ["no output"]
+            return dict(library=LIBRARY_STICK, unavailable=tail[0][:200])
+        return json.loads(lines[-1])
+    except Exception as e:  # no such library, or it failed: report why, measure nothing
+        return dict(library=LIBRARY_STICK, unavailable=f"{type(e).__name__}: {e}"[:200])
+
+
+def run_library_stick(arg: str, reps: int) -> dict:
+    """Child side of library_stick."""
+    import vllm._custom_ops as ops  # imported here only: the measuring stick's library
+
+    import fp8_block_scaled_tma_b200 as dg
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            torch.cuda._sleep(200000)
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        return statistics.median(ts)
+
+    out = []
+    for item in arg.split(";"):
+        M, N, K = (int(x) for x in item.split(","))
+        g = torch.Generator(device="cuda")
+        g.manual_seed(M * 7 + N * 3 + K)
+        a = (torch.randn(M, K, device="cuda", generator=g) * 0.5).to(torch.float8_e4m3fn)
+        b = (torch.randn(N, K, device="cuda", generator=g) * 0.5).to(torch.float8_e4m3fn)
+        kb, nb = K // 128, (N + 127) // 128
+        sa = torch.rand(M, kb, device="cuda", generator=g) + 0.5
+        sb = torch.rand(nb, kb, device="cuda", generator=g) + 0.5
+        d = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        sfa = dg.sfa_mn_major(sa)
+        ours = lambda: dg.dg_gemm_fp8_fp8_bf16_nt(a.view(torch.uint8), sfa, b.view(torch.uint8), sb, d)
+        # the library's layouts: B as [K, N] column-major, A scales [M, K/128] M-contiguous,
+        # B scales [K/128, N/128] K-contiguous
+        sa_l = sa.t().contiguous().t()
+        theirs = lambda: ops.cutlass_scaled_mm(a, b.t(), sa_l, sb.t(), torch.bfloat16)
+        us_ours = timed(ours)
+        ref = d.float()
+        us_lib = timed(theirs)
+        diff = ((theirs().float() - ref).abs() / (ref.abs() + 1.0)).max().item()
+        fl = 2.0 * M * N * K
+        out.append(dict(shape=f"{M}x{N}x{K}", ours_us=us_ours, ours_tflops=fl / us_ours / 1e6,
+                        library_us=us_lib, library_tflops=fl / us_lib / 1e6,
+                        speedup=us_lib / us_ours, max_rel_diff=diff))
+    return dict(library=LIBRARY_STICK, shapes=out)
+
+
 def back_to_back(dg, dev, flush, gate_cycles: int, reps: int = 10) -> dict:
     """The whole step enqueued back to back (no event between GEMMs), L2 flushed before it,
     timed by one event pair: with programmatic dependent launch off and on.  Each kernel's
@@ -563,6 +638,13 @@ def run_ours(args, rank, world, local_rank):
     # e2e through the public API with host buffers
     if not args.no_e2e:
         out["e2e"] = run_e2e(dg, dev, gemms, args, world)
+    if rank == 0 and world == 1 and not args.no_library_stick:
+        big = sorted(shapes, key=lambda sh: -sh["us"])
+        picks = [(sh["M"], sh["N"], sh["K"]) for sh in big if sh["kind"] == "dense"][:1]
+        picks += [(sh["M"], sh["N"], sh["K"]) for sh in big
+                  if sh["kind"] == "dense" and sh["M"] <= 128 and (sh["M"], sh["N"], sh["K"]) not in picks][:1]
+        if picks:
+            out["library_stick"] = library_stick(picks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(gemms, budget_s=args.cpu_seconds)
     return out
@@ -904,6 +986,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph timing of memory-bound shapes")
     ap.add_argument("--no-cublas", action="store_true", help="skip the cuBLAS FP8 measuring stick")
+    ap.add_argument("--no-library-stick", action="store_true",
+                    help="skip the block-scaled FP8 library measuring stick")
+    ap.add_argument("--library-stick", default=None, help=argparse.SUPPRESS)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="dram bytes per launch of the dominant kernel from an ncu capture")
@@ -922,6 +1007,9 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
+        return
+    if args.library_stick:
+        print(json.dumps(run_library_stick(args.library_stick, args.steps)), flush=True)
         return
 
     if world > 1:
