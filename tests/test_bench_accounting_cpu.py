@@ -90,3 +90,32 @@ def test_traffic_reported_only_for_unchanged_kernel_sources(monkeypatch):
     assert bench.measured_traffic("k stale")[0] is None
     assert bench.measured_traffic("k unknown")[0] is None
     assert bench.measured_traffic("k stale", 789)[0] == 789
+
+
+def test_library_stick_reports_why_when_the_child_fails(monkeypatch):
+    """The library measuring stick runs in a child process; when that process fails (no GPU,
+    no library) the line carries the reason and no numbers, and a child's JSON is passed on."""
+    import subprocess
+    import types
+
+    def failing(*a, **k):
+        return types.SimpleNamespace(returncode=1, stdout="", stderr="ModuleNotFoundError: no vllm\n")
+    monkeypatch.setattr(subprocess, "run", failing)
+    r = bench.library_stick([(8192, 7168, 18432)])
+    assert r["unavailable"] == "ModuleNotFoundError: no vllm" and "shapes" not in r
+
+    def raising(*a, **k):
+        raise subprocess.TimeoutExpired(cmd="bench.py", timeout=300)
+    monkeypatch.setattr(subprocess, "run", raising)
+    assert "TimeoutExpired" in bench.library_stick([(64, 2112, 7168)])["unavailable"]
+
+    seen = {}
+
+    def ok(cmd, **k):
+        seen["arg"] = cmd[cmd.index("--library-stick") + 1]
+        return types.SimpleNamespace(returncode=0, stderr="",
+                                     stdout='noise\n{"library": "x", "shapes": [{"shape": "1x2x3"}]}\n')
+    monkeypatch.setattr(subprocess, "run", ok)
+    r = bench.library_stick([(8192, 7168, 18432), (64, 2112, 7168)])
+    assert seen["arg"] == "8192,7168,18432;64,2112,7168"
+    assert r["shapes"][0]["shape"] == "1x2x3"
